@@ -1,0 +1,457 @@
+"""Benchmark of the paged-decode hot path on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload llama8b]
+    python bench.py --impl reference ...      # the fp64 CPU oracle, timed
+
+One step = one decode iteration of a serving loop over the whole batch:
+host slot assignment for one new token per request (C++ allocator),
+copy-on-write copies if any, pa_reshape_and_cache of the new K/V, and
+pa_decode (main kernel + split-K merge) over every request's cache.
+
+Prints one JSON line.  ``value`` is KV-read GB/s of pa_decode's algorithmic
+bytes (sum of L*2*Hkv*D*2 plus q/out/table bytes) over the device time of
+the K timed steps with every input resident in HBM; ``e2e`` is the same
+metric with each step's host allocator call, host->device copies of its
+inputs from pinned memory and the device->host read of its output inside the
+timed region.  Weak scaling over GPUs: every rank runs its own batch (its
+own pool and allocator), no data-path collective.
+"""
+
+import argparse
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+import workloads  # noqa: E402
+
+METRIC = "paged-decode KV-read GB/s & % of HBM peak; decode seqs/s at Llama-3-8B shape"
+PEAKS_FALLBACK = {"hbm_gbs": 6650.0, "source": "fallback"}
+INPUT_SETS = 4  # distinct q/k/v sets cycled through the steps
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            p = json.load(f)
+        return {"hbm_gbs": float(p["hbm_gbs"]), "source": "measured"}
+    except Exception:
+        return dict(PEAKS_FALLBACK)
+
+
+# --------------------------------------------------------------------------
+# clocks during the timed region (NVML, polled from a thread)
+# --------------------------------------------------------------------------
+class ClockSampler:
+    REASONS = {
+        0x1: "gpu_idle", 0x2: "applications_clocks_setting", 0x4: "sw_power_cap",
+        0x8: "hw_slowdown", 0x10: "sync_boost", 0x20: "sw_thermal_slowdown",
+        0x40: "hw_thermal_slowdown", 0x80: "hw_power_brake_slowdown",
+    }
+
+    def __init__(self, device_index, period_s=0.002):
+        self.samples, self.reasons = [], set()
+        self.period = period_s
+        self._stop = threading.Event()
+        self.max_mhz = None
+        try:
+            import pynvml
+
+            pynvml.nvmlInit()
+            self.nv = pynvml
+            self.h = pynvml.nvmlDeviceGetHandleByIndex(device_index)
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self.h, pynvml.NVML_CLOCK_SM)
+        except Exception:
+            self.nv = None
+
+    def _poll(self):
+        while not self._stop.is_set():
+            self.sample()
+            time.sleep(self.period)
+
+    def sample(self):
+        if self.nv is None:
+            return
+        try:
+            self.samples.append(self.nv.nvmlDeviceGetClockInfo(self.h, self.nv.NVML_CLOCK_SM))
+            bits = self.nv.nvmlDeviceGetCurrentClocksEventReasons(self.h)
+            for mask, name in self.REASONS.items():
+                if bits & mask and name != "gpu_idle":
+                    self.reasons.add(name)
+        except Exception:
+            pass
+
+    def __enter__(self):
+        self.sample()
+        self.t = threading.Thread(target=self._poll, daemon=True)
+        self.t.start()
+        return self
+
+    def __exit__(self, *exc):
+        self._stop.set()
+        self.t.join()
+
+    def summary(self):
+        if not self.samples:
+            return {"sm_mhz": None, "sm_max_mhz": self.max_mhz, "reasons": ["nvml unavailable"]}
+        return {"sm_mhz": statistics.median(self.samples), "sm_max_mhz": self.max_mhz,
+                "reasons": sorted(self.reasons), "samples": len(self.samples)}
+
+
+# --------------------------------------------------------------------------
+# workload state
+# --------------------------------------------------------------------------
+def decode_bytes(lens, hq, hkv, d, bs):
+    lens = np.asarray(lens, dtype=np.int64)
+    kv = int(lens.sum()) * 2 * hkv * d * 2
+    qo = 2 * len(lens) * hq * d * 2
+    tables = int((-(-lens // bs)).sum()) * 4 + len(lens) * 4
+    return kv + qo + tables, kv
+
+
+def build_cache(name, steps_total, rank, device):
+    import torch
+
+    from paged_kv_cache_354_b200.engine import PagedDecodeCache
+
+    p = workloads.plan(name, extra_tokens=steps_total + 1)
+    s = p.shape
+    lens0 = np.asarray(p.seq_lens, dtype=np.int64)
+    max_len = int(lens0.max()) + (p.prefix_len and 256) + steps_total + 2
+    batch = len(lens0) * (p.beams or 1)
+    cache = PagedDecodeCache(p.num_blocks, s.num_q_heads, s.num_kv_heads, s.head_dim, s.block_size,
+                             batch, max_len, initial_order=p.initial_order, device=device)
+    # pool content: bf16 N(0,1) from a seeded device generator (rank-distinct)
+    gen = torch.Generator(device=device)
+    gen.manual_seed(workloads.seed_of(name) * 1000 + rank)
+    cache.pool.copy_(torch.randn(cache.pool.shape, generator=gen, device=device,
+                                 dtype=torch.float32).to(torch.bfloat16))
+    ids = workloads.populate(cache.alloc, p)
+    if p.name == "beam":  # the 256 divergent tokens per beam go in before the decode loop
+        slots, pairs = cache.alloc.append_batch(ids, p.append_tokens, as_numpy=True)
+        k = torch.randn((len(slots), s.num_kv_heads, s.head_dim), generator=gen, device=device).bfloat16()
+        v = torch.randn((len(slots), s.num_kv_heads, s.head_dim), generator=gen, device=device).bfloat16()
+        from paged_kv_cache_354_b200 import pa_copy_blocks, pa_reshape_and_cache
+
+        pa_copy_blocks(cache.pool, torch.as_tensor(pairs, device=device))
+        pa_reshape_and_cache(k, v, cache.pool, torch.as_tensor(slots, device=device))
+    return p, cache, ids, gen
+
+
+def make_inputs(cache, batch, gen, device):
+    import torch
+
+    qs = [torch.randn((batch, cache.hq, cache.d), generator=gen, device=device).bfloat16()
+          for _ in range(INPUT_SETS)]
+    ks = [torch.randn((batch, cache.hkv, cache.d), generator=gen, device=device).bfloat16()
+          for _ in range(INPUT_SETS)]
+    vs = [torch.randn((batch, cache.hkv, cache.d), generator=gen, device=device).bfloat16()
+          for _ in range(INPUT_SETS)]
+    return qs, ks, vs
+
+
+# --------------------------------------------------------------------------
+# the GPU arm
+# --------------------------------------------------------------------------
+def run_gpu(args):
+    import torch
+    import torch.distributed as dist
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=__import__("datetime").timedelta(seconds=120))
+    device = torch.device("cuda", local if world > 1 else torch.cuda.current_device())
+    torch.cuda.set_device(device)
+    from paged_kv_cache_354_b200 import pa_device_error
+
+    K, W = args.steps, args.warmup
+    p, cache, ids, gen = build_cache(args.workload, 2 * (W + K), rank, device)
+    batch = len(ids)
+    qs, ks, vs = make_inputs(cache, batch, gen, device)
+    out = torch.empty_like(qs[0])
+    stream = torch.cuda.current_stream()
+
+    # ---- device-timed arm: all step metadata precomputed and resident
+    plans = [cache.plan_append(ids) for _ in range(W + K)]
+    d_slots = [torch.as_tensor(pl[0], device=device) for pl in plans]
+    d_pairs = [torch.as_tensor(pl[1].reshape(-1, 2), device=device) for pl in plans]
+    d_tables = [torch.as_tensor(pl[2], device=device) for pl in plans]
+    d_lens = [torch.as_tensor(pl[3], device=device) for pl in plans]
+    step_bytes = [decode_bytes(pl[3], cache.hq, cache.hkv, cache.d, cache.bs) for pl in plans]
+    launches = sum(cache.launches_per_step(len(pl[1])) for pl in plans[W:])
+
+    def dev_step(i):
+        j = i % INPUT_SETS
+        cache.run(qs[j], ks[j], vs[j], out, d_slots[i], d_tables[i], d_lens[i], d_pairs[i])
+
+    for i in range(W):
+        dev_step(i)
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(K)]
+    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with ClockSampler(device.index) as clocks:
+        start.record(stream)
+        for i in range(W, W + K):
+            j = i % INPUT_SETS
+            if d_pairs[i].shape[0]:
+                from paged_kv_cache_354_b200 import pa_copy_blocks
+
+                pa_copy_blocks(cache.pool, d_pairs[i])
+            from paged_kv_cache_354_b200 import pa_reshape_and_cache
+
+            pa_reshape_and_cache(ks[j], vs[j], cache.pool, d_slots[i])
+            ev[i - W][0].record(stream)
+            cache.decode(qs[j], out, d_tables[i], d_lens[i])
+            ev[i - W][1].record(stream)
+        end.record(stream)
+        torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    dev_ms = start.elapsed_time(end)
+    decode_ms = [a.elapsed_time(b) for a, b in ev]
+    bytes_timed = sum(b for b, _ in step_bytes[W:])
+    kv_timed = sum(kv for _, kv in step_bytes[W:])
+
+    # ---- end-to-end arm: host allocator + pinned H2D + kernels + D2H per step
+    h_q = [t.cpu().pin_memory() for t in qs]
+    h_k = [t.cpu().pin_memory() for t in ks]
+    h_v = [t.cpu().pin_memory() for t in vs]
+    d_q, d_k, d_v = torch.empty_like(qs[0]), torch.empty_like(ks[0]), torch.empty_like(vs[0])
+    h_out = torch.empty(out.shape, dtype=out.dtype).pin_memory()
+    e2e_bytes, e2e_h2d = 0, 0
+
+    def e2e_step(i):
+        nonlocal e2e_bytes, e2e_h2d
+        j = i % INPUT_SETS
+        slots, pairs, tables, lens = cache.plan_append(ids)
+        npairs = cache.stage(slots, pairs, tables, lens)
+        d_q.copy_(h_q[j], non_blocking=True)
+        d_k.copy_(h_k[j], non_blocking=True)
+        d_v.copy_(h_v[j], non_blocking=True)
+        cache.run(d_q, d_k, d_v, out, cache.d_slots[:batch], cache.d_tables[:batch], cache.d_lens[:batch],
+                  cache.d_pairs[:npairs])
+        h_out.copy_(out, non_blocking=True)
+        torch.cuda.current_stream().synchronize()
+        return decode_bytes(lens, cache.hq, cache.hkv, cache.d, cache.bs)[0], (
+            slots.nbytes + tables.nbytes + lens.nbytes + 8 * npairs + h_q[j].nbytes + 2 * h_k[j].nbytes)
+
+    for i in range(W):
+        e2e_step(i)
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    e_start, e_end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e_start.record(stream)
+    for i in range(K):
+        nb, h2d = e2e_step(W + i)
+        e2e_bytes += nb
+        e2e_h2d += h2d
+    e_end.record(stream)
+    torch.cuda.synchronize()
+    e2e_ms = e_start.elapsed_time(e_end)
+    dev_err = pa_device_error()
+
+    # ---- max over ranks
+    times = torch.tensor([dev_ms, e2e_ms, float(np.mean(decode_ms))], device=device, dtype=torch.float64)
+    totals = torch.tensor([bytes_timed, e2e_bytes, kv_timed], device=device, dtype=torch.float64)
+    if world > 1:
+        dist.all_reduce(times, op=dist.ReduceOp.MAX)
+        dist.all_reduce(totals, op=dist.ReduceOp.SUM)
+    dev_ms, e2e_ms, decode_avg_ms = times.tolist()
+    bytes_all, e2e_bytes_all, kv_all = totals.tolist()
+
+    if rank == 0:
+        peaks = load_peaks()
+        gbs = bytes_all / (dev_ms * 1e-3) / 1e9
+        per_launch_bytes = bytes_timed / K
+        achieved = per_launch_bytes / (decode_avg_ms * 1e-3) / 1e9
+        line = {
+            "metric": METRIC,
+            "value": round(gbs, 2),
+            "unit": "GB/s",
+            "n_gpus": world,
+            "steps": K,
+            "warmup": W,
+            "ms_per_step": round(dev_ms / K, 5),
+            "higher_is_better": True,
+            "scaling": "weak",
+            "vs_baseline": None,
+            "dtype": "bf16",
+            "data": "synthetic (seeded bf16 N(0,1) q/K/V; seeded lengths and shuffled block pool)",
+            "config": {
+                "workload": f"{args.workload}: B{batch} Hq{cache.hq}/Hkv{cache.hkv} D{cache.d} bs{cache.bs}",
+                "batch": batch, "num_q_heads": cache.hq, "num_kv_heads": cache.hkv, "head_dim": cache.d,
+                "block_size": cache.bs, "num_blocks": cache.num_blocks,
+                "mean_seq_len": round(float(np.mean(plans[W][3])), 1),
+                "split_k_partitions": cache.num_partitions,
+                "l2": f"inputs larger than L2: KV read per step {step_bytes[W][1] / 1e6:.0f} MB > 126 MB",
+                "parallelism": f"dp{world} (independent batches, no collective)",
+            },
+            "decode_seqs_per_s": round(batch * world * K / (dev_ms * 1e-3), 1),
+            "frac_of_hbm_peak": round(gbs / world / peaks["hbm_gbs"], 4),
+            "roofline": {
+                "bound": "hbm",
+                "kernel": "pa_decode (main + split-K merge)",
+                "achieved": round(achieved, 2),
+                "peak": peaks["hbm_gbs"],
+                "unit": "GB/s",
+                "frac": round(achieved / peaks["hbm_gbs"], 4),
+                "peak_source": peaks["source"],
+                "traffic": None,
+            },
+            "e2e": {
+                "value": round(e2e_bytes_all / (e2e_ms * 1e-3) / 1e9, 2),
+                "unit": "GB/s",
+                "h2d_bytes_per_step": int(e2e_h2d / K),
+                "d2h_bytes_per_step": int(h_out.nbytes),
+                "ms_per_step": round(e2e_ms / K, 5),
+            },
+            "gpu_launches": launches,
+            "clocks": clocks.summary(),
+            "device_error_word": dev_err,
+        }
+        if world == 1 and not args.no_cpu_baseline:
+            line["cpu_baseline"] = cpu_baseline(args.workload, args.cpu_seconds)
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+
+
+# --------------------------------------------------------------------------
+# the oracle on host cores
+# --------------------------------------------------------------------------
+class OracleRunner:
+    """The fp64 oracle decoding whole requests of a workload, one at a time.
+
+    The requests' tables come from the oracle's own allocator model; their
+    K/V blocks and queries are seeded bf16 N(0,1), built on the host outside
+    the timed part.  Only the oracle decode call is timed.
+    """
+
+    def __init__(self, name):
+        from oracle.block_allocator import BlockAllocator
+
+        self.name = name
+        p = workloads.plan(name)
+        self.shape = p.shape
+        self.alloc = BlockAllocator(p.num_blocks, p.shape.block_size, p.initial_order)
+        self.ids = workloads.populate(self.alloc, p)
+        self.order = np.random.default_rng(workloads.seed_of(name)).permutation(len(self.ids))
+        self.next = 0
+
+    def _request(self):
+        s = self.shape
+        sid = self.ids[self.order[self.next % len(self.ids)]]
+        self.next += 1
+        table = self.alloc.block_table(sid)
+        n = self.alloc.seq_len(sid)
+        blocks = workloads.bf16_normal((len(table), 2, s.num_kv_heads, s.block_size, s.head_dim),
+                                       seed=int(sid) + 1).double().numpy()
+        q = workloads.bf16_normal((1, s.num_q_heads, s.head_dim), seed=int(sid) + 7).double().numpy()
+        return q, blocks, np.arange(len(table))[None, :], n
+
+    def run(self, budget_s, min_requests=1):
+        """Decode requests until budget_s of oracle time; (kv_bytes, requests, seconds)."""
+        from threadpoolctl import threadpool_limits
+
+        from oracle import paged_attention as opa
+
+        s = self.shape
+        kv_bytes, done, elapsed = 0, 0, 0.0
+        with threadpool_limits(1):
+            while done < min_requests or elapsed < budget_s:
+                q, blocks, table, n = self._request()
+                t0 = time.perf_counter()
+                opa.decode(q, blocks, table, np.array([n]), 1.0 / math.sqrt(s.head_dim))
+                elapsed += time.perf_counter() - t0
+                kv_bytes += n * 2 * s.num_kv_heads * s.head_dim * 2
+                done += 1
+        return kv_bytes, done, elapsed
+
+    def describe(self, requests):
+        s = self.shape
+        return (f"{requests} whole requests of the {self.name} workload (all {s.num_q_heads} query heads "
+                f"each), fp64 NumPy oracle, 1 thread")
+
+
+def cpu_baseline(name, budget_s):
+    runner = OracleRunner(name)
+    kv, n, el = runner.run(budget_s)
+    return {"value": round(kv / el / 1e9, 4), "unit": "GB/s", "cores": 1, "kind": "oracle",
+            "sample": runner.describe(n), "seqs_per_s": round(n / el, 3),
+            "host_cores_available": len(os.sched_getaffinity(0))}
+
+
+def run_reference(args):
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return
+    runner = OracleRunner(args.workload)
+    per_step = args.cpu_seconds / max(1, args.steps + args.warmup)
+    for _ in range(args.warmup):
+        runner.run(per_step)
+    kv, n, el = 0, 0, 0.0
+    for _ in range(args.steps):
+        a, b, c = runner.run(per_step)
+        kv, n, el = kv + a, n + b, el + c
+    value = kv / el / 1e9
+    line = {
+        "impl": "reference",
+        "metric": METRIC,
+        "value": round(value, 4),
+        "unit": "GB/s",
+        "n_gpus": int(os.environ.get("WORLD_SIZE", "1")),
+        "steps": args.steps,
+        "warmup": args.warmup,
+        "ms_per_step": round(1e3 * el / args.steps, 3),
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "f64",
+        "data": "synthetic (seeded bf16 N(0,1) K/V and q, upcast to f64)",
+        "config": {"workload": args.workload,
+                   "note": "each step decodes at least one whole request of the workload on the host"},
+        "cpu_baseline": {"value": round(value, 4), "unit": "GB/s", "cores": 1, "kind": "oracle",
+                         "sample": runner.describe(n)},
+        "e2e": {"value": round(value, 4), "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+def main():
+    ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--workload", default="llama8b", choices=workloads.NAMES)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--cpu-seconds", type=float, default=10.0)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        ap.error("--warmup must be at least 3")
+    if args.impl == "reference":
+        run_reference(args)
+    else:
+        run_gpu(args)
+
+
+if __name__ == "__main__":
+    main()

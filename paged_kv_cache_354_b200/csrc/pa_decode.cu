@@ -1,0 +1,869 @@
+// pa_decode: single-token decode attention over the paged KV pool.
+//
+// What it computes is the quiz page's sketch ("Conceptual: PagedAttention
+// block lookup"): for each request b and query head j, keys and values of
+// logical position pos come from physical block block_table[b][pos / bs],
+// row pos % bs, followed by scaled-dot-product attention.  The sketch notes
+// that real kernels fold the gather into the inner tiling loop; here the
+// gather *is* the tiling loop: one tile = one physical block of one KV head.
+//
+// Design for sm_100a (one CTA per (request, KV head, sequence partition)):
+//  * a producer warp reads the partition's block-table entries and issues
+//    one TMA tile load per physical block and 64-dim slab (box 64 x bs x 2
+//    covers the K rows and the V rows of that block and head), into a
+//    multi-stage shared-memory ring with 128-byte swizzle, completion on
+//    mbarriers;
+//  * four consumer warps each own every fourth block and keep their own
+//    online-softmax state; the query heads of a GQA group share every loaded
+//    tile;
+//  * consumer math: for groups >= 4 (and on request) bf16 mma.sync with
+//    fp32 accumulate in a transposed form, S^T = K Q^T then O^T += V^T P^T,
+//    so the 16-row side of the MMA is the token / head-dim axis and the
+//    group of g <= 8 query heads fills the 8-wide side; P^T is formed from
+//    the S^T accumulators in registers with movmatrix.  For groups <= 2,
+//    fp32 FMA on CUDA cores;
+//  * the warps' partial states merge through shared memory; a sequence cut
+//    into several partitions writes fp32 partials (O, running max, sum) and
+//    a second kernel merges them with the log-sum-exp rule.
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+
+#include <cmath>
+
+#include "pa_device.cuh"
+#include "pa_internal.h"
+
+namespace pa {
+
+constexpr int kConsumerWarps = 4;
+constexpr int kThreads = (kConsumerWarps + 1) * 32;
+constexpr int kMaxGroup = 8;
+constexpr unsigned kFull = 0xffffffffu;
+
+enum Variant { kCudaCore = 1, kMma = 2 };
+
+template <int D, int BS>
+struct Geo {
+  static_assert(D % 64 == 0, "head_dim must be a multiple of 64");
+  static_assert(BS % 16 == 0, "block_size must be a multiple of 16");
+  static constexpr int kRegions = D / 64;                  // 64-dim slabs of a row
+  static constexpr int kRegionBytes = 2 * BS * 128;        // K rows then V rows of one slab
+  static constexpr int kStageBytes = kRegions * kRegionBytes;  // one block of one head
+  static constexpr int kStages = (kStageBytes <= 8192) ? 8 : 4;
+  static constexpr int kStageSmem = kStages * kStageBytes;
+  static_assert(kStages % kConsumerWarps == 0, "stage s must always go to warp s % warps");
+  // epilogue scratch aliased on the stage ring
+  static constexpr int kEpiO = kConsumerWarps * kMaxGroup * D * 4;
+  static constexpr int kEpiBytes = kEpiO + 2 * kConsumerWarps * kMaxGroup * 4;
+  static_assert(kEpiBytes <= kStageSmem, "epilogue scratch must fit in the stage ring");
+};
+
+// Shared-memory carve-up after the 1024-byte aligned stage ring.
+template <int D, int BS, int G>
+struct Smem {
+  using geo = Geo<D, BS>;
+  static constexpr int kBar = geo::kStageSmem;                          // full[S], empty[S]
+  static constexpr int kMisc = kBar + 16 * geo::kStages;                // last_round[S], abort
+  static constexpr int kPbuf = (kMisc + 4 * geo::kStages + 4 + 15) & ~15;  // CUDA-core p tiles
+  static constexpr int kPbufBytes = kConsumerWarps * BS * (G > 0 ? G : 1) * 4;
+  static constexpr int kFw = kPbuf + kPbufBytes;                        // merge factors
+  static constexpr int kTotal = kFw + (kConsumerWarps * kMaxGroup + 2 * kMaxGroup) * 4;
+  static constexpr int kDynamic = kTotal + 1024;                        // alignment slack
+};
+
+struct DecodeArgs {
+  __nv_bfloat16* out;
+  const __nv_bfloat16* q;
+  const int32_t* block_tables;
+  const int32_t* seq_lens;
+  float* part_o;  // [B*Hq][max_parts][D]
+  float* part_m;  // [B*Hq][max_parts]
+  float* part_l;  // [B*Hq][max_parts]
+  int32_t* err;
+  int num_q_heads, num_kv_heads, group;
+  int num_blocks, max_blocks_per_seq;
+  int part_blocks, max_parts;
+  float scale_log2;  // scale * log2(e)
+};
+
+// Tokens of request b the kernels attend over, after the device-side checks
+// (both kernels use this, so they agree on the partition count).
+__device__ __forceinline__ int effective_len(int raw, int bs, const DecodeArgs& a, bool report) {
+  int len = raw < 0 ? 0 : raw;
+  const int cap_table = a.max_blocks_per_seq * bs;
+  const long long cap_grid = static_cast<long long>(a.max_parts) * a.part_blocks * bs;
+  if (len > cap_table || len > cap_grid || raw < 0) {
+    if (report) flag_error(a.err, PA_DEVERR_SEQ_LEN);
+    len = min(len, cap_table);
+    len = static_cast<int>(min(static_cast<long long>(len), cap_grid));
+  }
+  return len;
+}
+
+// --------------------------------------------------------------------------
+// Tensor-core consumer: state and per-block step.
+// --------------------------------------------------------------------------
+template <int D, int BS>
+struct MmaConsumer {
+  using geo = Geo<D, BS>;
+  static constexpr int kDT = D / 16;   // 16-dim tiles of the head dim
+  static constexpr int kTT = BS / 16;  // 16-token tiles of a block
+  uint32_t qb[kDT][2];                 // Q^T as the B operand of S^T = K Q^T
+  float o[kDT][4];                     // O^T accumulators
+  float m0, m1, l0, l1;                // two head columns of this thread
+
+  __device__ __forceinline__ void init(const __nv_bfloat16* qrow_base, int group, int lane) {
+    const int head = lane >> 2;
+    const int c = 2 * (lane & 3);
+#pragma unroll
+    for (int ks = 0; ks < kDT; ++ks) {
+      if (head < group) {
+        const __nv_bfloat16* qr = qrow_base + head * D + 16 * ks + c;
+        qb[ks][0] = *reinterpret_cast<const uint32_t*>(qr);
+        qb[ks][1] = *reinterpret_cast<const uint32_t*>(qr + 8);
+      } else {
+        qb[ks][0] = 0u;
+        qb[ks][1] = 0u;
+      }
+    }
+#pragma unroll
+    for (int dt = 0; dt < kDT; ++dt) o[dt][0] = o[dt][1] = o[dt][2] = o[dt][3] = 0.f;
+    m0 = m1 = -INFINITY;
+    l0 = l1 = 0.f;
+  }
+
+  __device__ __forceinline__ void step(uint32_t sb, int valid, float scale_log2, int lane) {
+    const int mat = lane >> 3;
+    const int r8 = lane & 7;
+    // ---- S^T = K Q^T : rows = tokens, cols = query heads of the group
+    float s[kTT][4];
+#pragma unroll
+    for (int mt = 0; mt < kTT; ++mt) {
+      s[mt][0] = s[mt][1] = s[mt][2] = s[mt][3] = 0.f;
+      const int tok = 16 * mt + ((mat & 1) << 3) + r8;
+#pragma unroll
+      for (int ks = 0; ks < kDT; ++ks) {
+        const int chunk = (2 * (ks & 3) + (mat >> 1)) ^ r8;
+        const uint32_t addr = sb + (ks >> 2) * geo::kRegionBytes + tok * 128 + chunk * 16;
+        uint32_t a0, a1, a2, a3;
+        ldsm_x4(addr, a0, a1, a2, a3);
+        mma_bf16_16816(s[mt], a0, a1, a2, a3, qb[ks][0], qb[ks][1]);
+      }
+    }
+    // ---- scale, mask rows past the request's end, column max
+    float mx0 = -INFINITY, mx1 = -INFINITY;
+#pragma unroll
+    for (int mt = 0; mt < kTT; ++mt) {
+      const int t0 = 16 * mt + (lane >> 2);
+      const bool ok0 = t0 < valid, ok1 = t0 + 8 < valid;
+      s[mt][0] = ok0 ? s[mt][0] * scale_log2 : -INFINITY;
+      s[mt][1] = ok0 ? s[mt][1] * scale_log2 : -INFINITY;
+      s[mt][2] = ok1 ? s[mt][2] * scale_log2 : -INFINITY;
+      s[mt][3] = ok1 ? s[mt][3] * scale_log2 : -INFINITY;
+      mx0 = fmaxf(mx0, fmaxf(s[mt][0], s[mt][2]));
+      mx1 = fmaxf(mx1, fmaxf(s[mt][1], s[mt][3]));
+    }
+#pragma unroll
+    for (int off = 4; off < 32; off <<= 1) {
+      mx0 = fmaxf(mx0, __shfl_xor_sync(kFull, mx0, off));
+      mx1 = fmaxf(mx1, __shfl_xor_sync(kFull, mx1, off));
+    }
+    const float n0 = fmaxf(m0, mx0), n1 = fmaxf(m1, mx1);
+    // rescale only when some column's running max moved (warp-uniform test)
+    if (__any_sync(kFull, (n0 > m0) || (n1 > m1))) {
+      const float a0 = (m0 == -INFINITY) ? 0.f : exp2f(m0 - n0);
+      const float a1 = (m1 == -INFINITY) ? 0.f : exp2f(m1 - n1);
+#pragma unroll
+      for (int dt = 0; dt < kDT; ++dt) {
+        o[dt][0] *= a0;
+        o[dt][2] *= a0;
+        o[dt][1] *= a1;
+        o[dt][3] *= a1;
+      }
+      l0 *= a0;
+      l1 *= a1;
+      m0 = n0;
+      m1 = n1;
+    }
+    // ---- P (bf16) -> P^T fragments; O^T += V^T P^T
+#pragma unroll
+    for (int mt = 0; mt < kTT; ++mt) {
+      const uint32_t pa = pack_bf16x2(exp2f(s[mt][0] - m0), exp2f(s[mt][1] - m1));
+      const uint32_t pb = pack_bf16x2(exp2f(s[mt][2] - m0), exp2f(s[mt][3] - m1));
+      l0 += bf16lo_to_f32(pa) + bf16lo_to_f32(pb);
+      l1 += bf16hi_to_f32(pa) + bf16hi_to_f32(pb);
+      const uint32_t b0 = movmatrix_trans(pa);
+      const uint32_t b1 = movmatrix_trans(pb);
+      const int row = BS + 16 * mt + ((mat >> 1) << 3) + r8;
+#pragma unroll
+      for (int dt = 0; dt < kDT; ++dt) {
+        const int chunk = (2 * (dt & 3) + (mat & 1)) ^ r8;
+        const uint32_t addr = sb + (dt >> 2) * geo::kRegionBytes + row * 128 + chunk * 16;
+        uint32_t a0, a1, a2, a3;
+        ldsm_x4_trans(addr, a0, a1, a2, a3);
+        mma_bf16_16816(o[dt], a0, a1, a2, a3, b0, b1);
+      }
+    }
+  }
+
+  // Write this warp's unnormalised O, running max and sum to the epilogue
+  // scratch: o_s[head][dim], m_s[head], l_s[head].
+  __device__ __forceinline__ void store(float* o_s, float* m_s, float* l_s, int lane) {
+#pragma unroll
+    for (int off = 4; off < 32; off <<= 1) {
+      l0 += __shfl_xor_sync(kFull, l0, off);
+      l1 += __shfl_xor_sync(kFull, l1, off);
+    }
+    const int h0 = 2 * (lane & 3);
+#pragma unroll
+    for (int dt = 0; dt < kDT; ++dt) {
+      const int d = 16 * dt + (lane >> 2);
+      o_s[h0 * D + d] = o[dt][0];
+      o_s[(h0 + 1) * D + d] = o[dt][1];
+      o_s[h0 * D + d + 8] = o[dt][2];
+      o_s[(h0 + 1) * D + d + 8] = o[dt][3];
+    }
+    if (lane < 4) {
+      m_s[h0] = m0;
+      m_s[h0 + 1] = m1;
+      l_s[h0] = l0;
+      l_s[h0 + 1] = l1;
+    }
+  }
+};
+
+// --------------------------------------------------------------------------
+// CUDA-core consumer for narrow groups (G query heads per KV head).
+// QK: a quad of 4 lanes per token, 8 tokens per pass, the quad splits the
+//     head dim; PV: each lane owns D/32 consecutive output dims.
+// --------------------------------------------------------------------------
+template <int D, int BS, int G>
+struct CudaCoreConsumer {
+  using geo = Geo<D, BS>;
+  static constexpr int kQD = D / 4;     // dims per lane in QK
+  static constexpr int kPass = BS / 8;  // token passes per block
+  static constexpr int kOD = D / 32;    // output dims per lane in PV
+  float qf[G][kQD];
+  float o[G][kOD];
+  float m[G], l[G];
+
+  __device__ __forceinline__ void init(const __nv_bfloat16* qrow_base, int lane) {
+    const int qq = lane & 3;
+#pragma unroll
+    for (int j = 0; j < G; ++j) {
+#pragma unroll
+      for (int x = 0; x < D / 64; ++x)
+#pragma unroll
+        for (int hi = 0; hi < 2; ++hi) {
+          const int d0 = x * 64 + (qq + 4 * hi) * 8;
+          const uint4 raw = *reinterpret_cast<const uint4*>(qrow_base + j * D + d0);
+          const uint32_t w[4] = {raw.x, raw.y, raw.z, raw.w};
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            qf[j][(x * 2 + hi) * 8 + 2 * e] = bf16lo_to_f32(w[e]);
+            qf[j][(x * 2 + hi) * 8 + 2 * e + 1] = bf16hi_to_f32(w[e]);
+          }
+        }
+#pragma unroll
+      for (int e = 0; e < kOD; ++e) o[j][e] = 0.f;
+      m[j] = -INFINITY;
+      l[j] = 0.f;
+    }
+  }
+
+  __device__ __forceinline__ void step(uint32_t sb, float* pbuf, int valid, float scale_log2,
+                                       int lane) {
+    const int qq = lane & 3;
+    const int qd = lane >> 2;
+    float s[kPass][G];
+#pragma unroll
+    for (int ps = 0; ps < kPass; ++ps) {
+      // quads (2k, 2k+1) take tokens (k, k+4): conflict-free 16-byte reads
+      const int tok = ps * 8 + ((qd & 1) << 2) + (qd >> 1);
+      float dot[G];
+#pragma unroll
+      for (int j = 0; j < G; ++j) dot[j] = 0.f;
+#pragma unroll
+      for (int x = 0; x < D / 64; ++x)
+#pragma unroll
+        for (int hi = 0; hi < 2; ++hi) {
+          const int chunk = (qq + 4 * hi) ^ (tok & 7);
+          uint4 raw;
+          asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];"
+                       : "=r"(raw.x), "=r"(raw.y), "=r"(raw.z), "=r"(raw.w)
+                       : "r"(sb + x * geo::kRegionBytes + tok * 128 + chunk * 16));
+          const uint32_t w[4] = {raw.x, raw.y, raw.z, raw.w};
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            const float k0 = bf16lo_to_f32(w[e]), k1 = bf16hi_to_f32(w[e]);
+#pragma unroll
+            for (int j = 0; j < G; ++j) {
+              dot[j] = fmaf(k0, qf[j][(x * 2 + hi) * 8 + 2 * e], dot[j]);
+              dot[j] = fmaf(k1, qf[j][(x * 2 + hi) * 8 + 2 * e + 1], dot[j]);
+            }
+          }
+        }
+#pragma unroll
+      for (int j = 0; j < G; ++j) {
+        dot[j] += __shfl_xor_sync(kFull, dot[j], 1);
+        dot[j] += __shfl_xor_sync(kFull, dot[j], 2);
+        s[ps][j] = tok < valid ? dot[j] * scale_log2 : -INFINITY;
+      }
+    }
+    float mx[G];
+    bool moved = false;
+#pragma unroll
+    for (int j = 0; j < G; ++j) {
+      mx[j] = s[0][j];
+#pragma unroll
+      for (int ps = 1; ps < kPass; ++ps) mx[j] = fmaxf(mx[j], s[ps][j]);
+#pragma unroll
+      for (int off = 4; off < 32; off <<= 1) mx[j] = fmaxf(mx[j], __shfl_xor_sync(kFull, mx[j], off));
+      mx[j] = fmaxf(mx[j], m[j]);
+      moved |= mx[j] > m[j];
+    }
+    if (__any_sync(kFull, moved)) {  // values are warp-uniform; the vote keeps it explicit
+#pragma unroll
+      for (int j = 0; j < G; ++j) {
+        const float a = (m[j] == -INFINITY) ? 0.f : exp2f(m[j] - mx[j]);
+#pragma unroll
+        for (int e = 0; e < kOD; ++e) o[j][e] *= a;
+        l[j] *= a;
+        m[j] = mx[j];
+      }
+    }
+#pragma unroll
+    for (int ps = 0; ps < kPass; ++ps) {
+      const int tok = ps * 8 + ((qd & 1) << 2) + (qd >> 1);
+#pragma unroll
+      for (int j = 0; j < G; ++j) {
+        const float p = exp2f(s[ps][j] - m[j]);
+        l[j] += p;
+        if (qq == 0) pbuf[tok * G + j] = p;
+      }
+    }
+    __syncwarp();
+    // ---- PV over the valid rows only (rows past the end may hold NaN)
+    const int x = (D == 128) ? (lane >> 4) : 0;
+    const int c = (D == 128) ? ((lane & 15) >> 1) : (lane >> 2);
+    const int sub = (D == 128) ? (lane & 1) * 8 : (lane & 3) * 4;
+#pragma unroll 4
+    for (int tok = 0; tok < valid; ++tok) {
+      const uint32_t addr =
+          sb + x * geo::kRegionBytes + (BS + tok) * 128 + ((c ^ (tok & 7)) << 4) + sub;
+      float v[kOD];
+      if constexpr (kOD == 4) {
+        uint32_t w0, w1;
+        asm volatile("ld.shared.v2.u32 {%0, %1}, [%2];" : "=r"(w0), "=r"(w1) : "r"(addr));
+        v[0] = bf16lo_to_f32(w0);
+        v[1] = bf16hi_to_f32(w0);
+        v[2] = bf16lo_to_f32(w1);
+        v[3] = bf16hi_to_f32(w1);
+      } else {
+        uint32_t w0;
+        asm volatile("ld.shared.u32 %0, [%1];" : "=r"(w0) : "r"(addr));
+        v[0] = bf16lo_to_f32(w0);
+        v[1] = bf16hi_to_f32(w0);
+      }
+#pragma unroll
+      for (int j = 0; j < G; ++j) {
+        const float p = pbuf[tok * G + j];
+#pragma unroll
+        for (int e = 0; e < kOD; ++e) o[j][e] = fmaf(p, v[e], o[j][e]);
+      }
+    }
+  }
+
+  __device__ __forceinline__ void store(float* o_s, float* m_s, float* l_s, int lane) {
+#pragma unroll
+    for (int j = 0; j < G; ++j) {
+      float lj = l[j];
+#pragma unroll
+      for (int off = 4; off < 32; off <<= 1) lj += __shfl_xor_sync(kFull, lj, off);
+#pragma unroll
+      for (int e = 0; e < kOD; ++e) o_s[j * D + lane * kOD + e] = o[j][e];
+      if (lane == 0) {
+        m_s[j] = m[j];
+        l_s[j] = lj;
+      }
+    }
+  }
+};
+
+// --------------------------------------------------------------------------
+// The decode kernel.  grid = (max_parts, num_kv_heads, batch).
+// --------------------------------------------------------------------------
+template <int D, int BS, int VAR, int G>
+__global__ void __launch_bounds__(kThreads, (VAR == kMma || G <= 2) ? 3 : 2)
+    paged_decode_kernel(const __grid_constant__ CUtensorMap kv_map, const DecodeArgs a) {
+  using geo = Geo<D, BS>;
+  using sm = Smem<D, BS, G>;
+  extern __shared__ uint8_t smem_raw[];
+  const uint32_t raw_base = smem_u32(smem_raw);
+  const uint32_t pad = ((raw_base + 1023u) & ~1023u) - raw_base;
+  uint8_t* smem = smem_raw + pad;
+  const uint32_t sbase = raw_base + pad;
+
+  const int part = blockIdx.x;
+  const int kvh = blockIdx.y;
+  const int b = blockIdx.z;
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const int g = a.group;
+
+  const int len = effective_len(__ldg(a.seq_lens + b), BS, a, part == 0 && threadIdx.x == 0);
+  const int nblk = (len + BS - 1) / BS;
+  const int nparts = (nblk + a.part_blocks - 1) / a.part_blocks;
+  const size_t head0 = static_cast<size_t>(b) * a.num_q_heads + static_cast<size_t>(kvh) * g;
+  if (len == 0) {  // nothing to attend over: output is zero
+    if (part == 0)
+      for (int i = threadIdx.x; i < g * D; i += kThreads)
+        a.out[head0 * D + i] = __float2bfloat16_rn(0.f);
+    return;
+  }
+  if (part >= nparts) return;
+  const int blk0 = part * a.part_blocks;
+  const int n = min(a.part_blocks, nblk - blk0);
+  const int last_valid = len - (nblk - 1) * BS;  // rows of the request's final block
+
+  const uint32_t bar_full = sbase + sm::kBar;
+  const uint32_t bar_empty = bar_full + 8 * geo::kStages;
+  int* last_round = reinterpret_cast<int*>(smem + sm::kMisc);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + sm::kMisc + 4 * geo::kStages);
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < geo::kStages; ++s) {
+      mbar_init(bar_full + 8 * s, 1);
+      mbar_init(bar_empty + 8 * s, 1);
+      last_round[s] = -1;
+    }
+    *abort_flag = 0;
+    fence_barrier_init();
+  }
+  __syncthreads();
+
+  [[maybe_unused]] MmaConsumer<D, BS> mc;
+  [[maybe_unused]] CudaCoreConsumer<D, BS, (G > 0 ? G : 1)> cc;
+  if (warp == kConsumerWarps) {
+    // ------------------------------------------------------------ producer
+    if (lane == 0) prefetch_tensor_map(&kv_map);
+    const int32_t* trow =
+        a.block_tables + static_cast<size_t>(b) * a.max_blocks_per_seq + blk0;
+    bool stop = false;
+    for (int base = 0; base < n && !stop; base += 32) {
+      int phys = 0;
+      if (base + lane < n) {
+        phys = __ldg(trow + base + lane);
+        if (static_cast<unsigned>(phys) >= static_cast<unsigned>(a.num_blocks)) {
+          flag_error(a.err, PA_DEVERR_BLOCK_ID);
+          phys = 0;  // read a valid block instead; the result is flagged as wrong
+        }
+      }
+      const int cnt = min(32, n - base);
+      for (int j = 0; j < cnt; ++j) {
+        const int pb = __shfl_sync(kFull, phys, j);
+        int failed = 0;
+        if (lane == 0) {
+          const int i = base + j;
+          const int s = i % geo::kStages;
+          const int round = i / geo::kStages;
+          if (!mbar_wait(bar_empty + 8 * s, (round & 1) ^ 1)) {
+            flag_error(a.err, PA_DEVERR_WAIT_TIMEOUT);
+            *abort_flag = 1;
+            failed = 1;
+          } else {
+            const uint32_t fb = bar_full + 8 * s;
+            mbar_arrive_expect_tx(fb, geo::kStageBytes);
+            const uint32_t dst = sbase + s * geo::kStageBytes;
+#pragma unroll
+            for (int x = 0; x < geo::kRegions; ++x)
+              tma_load_3d(dst + x * geo::kRegionBytes, &kv_map, fb, x * 64, kvh * BS, 2 * pb);
+            last_round[s] = round;
+          }
+        }
+        if (__shfl_sync(kFull, failed, 0)) {
+          stop = true;
+          break;
+        }
+      }
+    }
+  } else {
+    // ----------------------------------------------------------- consumers
+    const __nv_bfloat16* qrow = a.q + head0 * D;
+    float* pbuf = reinterpret_cast<float*>(smem + sm::kPbuf) + warp * BS * (G > 0 ? G : 1);
+    if constexpr (VAR == kMma) mc.init(qrow, g, lane);
+    else cc.init(qrow, lane);
+    for (int i = warp; i < n; i += kConsumerWarps) {
+      if (*abort_flag) break;
+      const int s = i % geo::kStages;
+      if (!mbar_wait(bar_full + 8 * s, (i / geo::kStages) & 1)) {
+        if (lane == 0) {
+          flag_error(a.err, PA_DEVERR_WAIT_TIMEOUT);
+          *abort_flag = 1;
+        }
+        break;
+      }
+      const uint32_t sb = sbase + s * geo::kStageBytes;
+      const int valid = (blk0 + i == nblk - 1) ? last_valid : BS;
+      if constexpr (VAR == kMma) {
+        if (valid < BS) {
+          // rows past the end may hold anything, even NaN: zero their V so
+          // that P = 0 there contributes exactly 0
+          const int rows = BS - valid;
+          for (int t = lane; t < rows * geo::kRegions * 8; t += 32) {
+            const int r = valid + t / (geo::kRegions * 8);
+            const int x = (t / 8) % geo::kRegions;
+            const int ch = t % 8;
+            asm volatile("st.shared.v4.u32 [%0], {%1, %1, %1, %1};" ::"r"(
+                             sb + x * geo::kRegionBytes + (BS + r) * 128 + ch * 16),
+                         "r"(0u)
+                         : "memory");
+          }
+          // order these generic writes before the next TMA refill of the stage
+          fence_proxy_async_smem();
+          __syncwarp();
+        }
+        mc.step(sb, valid, a.scale_log2, lane);
+      } else {
+        cc.step(sb, pbuf, valid, a.scale_log2, lane);
+      }
+      __syncwarp();
+      if (lane == 0) mbar_arrive(bar_empty + 8 * s);
+    }
+  }
+  __syncthreads();  // (A) the stage ring is idle; it becomes epilogue scratch
+  if (warp < kConsumerWarps && *abort_flag == 0) {
+    float* o_s = reinterpret_cast<float*>(smem) + warp * kMaxGroup * D;
+    float* m_s = reinterpret_cast<float*>(smem + geo::kEpiO) + warp * kMaxGroup;
+    float* l_s = m_s + kConsumerWarps * kMaxGroup;
+    if constexpr (VAR == kMma) mc.store(o_s, m_s, l_s, lane);
+    else cc.store(o_s, m_s, l_s, lane);
+  }
+  __syncthreads();  // (B) epilogue scratch written
+
+  if (*abort_flag) {
+    // unwind: let every issued tile land before the CTA's memory goes away
+    if (threadIdx.x == 0)
+      for (int s = 0; s < geo::kStages; ++s)
+        if (last_round[s] >= 0) mbar_wait_bounded(bar_full + 8 * s, last_round[s] & 1, kWaitLimitNs);
+    return;
+  }
+
+  // ---------------------------------------------------------- merge warps
+  const float* o_all = reinterpret_cast<const float*>(smem);
+  const float* m_all = reinterpret_cast<const float*>(smem + geo::kEpiO);
+  const float* l_all = m_all + kConsumerWarps * kMaxGroup;
+  float* fw = reinterpret_cast<float*>(smem + sm::kFw);  // [warp][head]
+  float* mrow = fw + kConsumerWarps * kMaxGroup;         // [head]
+  float* lrow = mrow + kMaxGroup;                        // [head]
+  const bool single = (nparts == 1);
+  if (threadIdx.x < g) {
+    const int j = threadIdx.x;
+    float mm = -INFINITY;
+    for (int w = 0; w < kConsumerWarps; ++w) mm = fmaxf(mm, m_all[w * kMaxGroup + j]);
+    float f[kConsumerWarps];
+    float ll = 0.f;
+    for (int w = 0; w < kConsumerWarps; ++w) {
+      const float mw = m_all[w * kMaxGroup + j];
+      f[w] = (mw == -INFINITY) ? 0.f : exp2f(mw - mm);
+      ll += f[w] * l_all[w * kMaxGroup + j];
+    }
+    const float inv = single ? 1.f / ll : 1.f;
+    for (int w = 0; w < kConsumerWarps; ++w) fw[w * kMaxGroup + j] = f[w] * inv;
+    mrow[j] = mm;
+    lrow[j] = ll;
+  }
+  __syncthreads();
+  for (int idx = threadIdx.x; idx < g * D / 2; idx += kThreads) {
+    const int j = (2 * idx) / D;
+    const int d = (2 * idx) % D;
+    float v0 = 0.f, v1 = 0.f;
+#pragma unroll
+    for (int w = 0; w < kConsumerWarps; ++w) {
+      const float f = fw[w * kMaxGroup + j];
+      const float* ow = o_all + (w * kMaxGroup + j) * D + d;
+      v0 = fmaf(f, ow[0], v0);
+      v1 = fmaf(f, ow[1], v1);
+    }
+    if (single) {
+      *reinterpret_cast<__nv_bfloat162*>(a.out + (head0 + j) * D + d) =
+          __floats2bfloat162_rn(v0, v1);
+    } else {
+      const size_t row = (head0 + j) * a.max_parts + part;
+      *reinterpret_cast<float2*>(a.part_o + row * D + d) = make_float2(v0, v1);
+      if (d == 0) {
+        a.part_m[row] = mrow[j];
+        a.part_l[row] = lrow[j];
+      }
+    }
+  }
+}
+
+// --------------------------------------------------------------------------
+// Log-sum-exp merge of the sequence partitions: one warp per (request, head).
+//   M = max_p m_p;  out = sum_p 2^(m_p - M) O_p / sum_p 2^(m_p - M) l_p
+// (m in the log2 domain; O_p unnormalised w.r.t. its own m_p).
+// --------------------------------------------------------------------------
+template <int D, int BS>
+__global__ void __launch_bounds__(128) paged_decode_reduce_kernel(const DecodeArgs a, int batch) {
+  constexpr int kPer = D / 32;
+  const int gw = blockIdx.x * 4 + (threadIdx.x >> 5);
+  const int lane = threadIdx.x & 31;
+  if (gw >= batch * a.num_q_heads) return;
+  const int b = gw / a.num_q_heads;
+  const int len = effective_len(__ldg(a.seq_lens + b), BS, a, false);
+  const int nblk = (len + BS - 1) / BS;
+  const int nparts = (nblk + a.part_blocks - 1) / a.part_blocks;
+  if (nparts <= 1) return;  // the main kernel wrote this output directly
+  const size_t base = static_cast<size_t>(gw) * a.max_parts;
+  float mm = -INFINITY;
+  for (int p = lane; p < nparts; p += 32) mm = fmaxf(mm, a.part_m[base + p]);
+#pragma unroll
+  for (int off = 16; off > 0; off >>= 1) mm = fmaxf(mm, __shfl_xor_sync(kFull, mm, off));
+  float acc[kPer];
+#pragma unroll
+  for (int e = 0; e < kPer; ++e) acc[e] = 0.f;
+  float den = 0.f;
+  for (int p = 0; p < nparts; ++p) {
+    const float w = exp2f(a.part_m[base + p] - mm);
+    den = fmaf(w, a.part_l[base + p], den);
+    const float* op = a.part_o + (base + p) * D + lane * kPer;
+    if constexpr (kPer == 4) {
+      const float4 v = *reinterpret_cast<const float4*>(op);
+      acc[0] = fmaf(w, v.x, acc[0]);
+      acc[1] = fmaf(w, v.y, acc[1]);
+      acc[2] = fmaf(w, v.z, acc[2]);
+      acc[3] = fmaf(w, v.w, acc[3]);
+    } else {
+      const float2 v = *reinterpret_cast<const float2*>(op);
+      acc[0] = fmaf(w, v.x, acc[0]);
+      acc[1] = fmaf(w, v.y, acc[1]);
+    }
+  }
+  const float inv = 1.f / den;
+  __nv_bfloat16* o = a.out + static_cast<size_t>(gw) * D + lane * kPer;
+#pragma unroll
+  for (int e = 0; e < kPer; e += 2)
+    *reinterpret_cast<__nv_bfloat162*>(o + e) = __floats2bfloat162_rn(acc[e] * inv, acc[e + 1] * inv);
+}
+
+// --------------------------------------------------------------------------
+// Host side
+// --------------------------------------------------------------------------
+struct Plan {
+  int part_blocks = 1;
+  int max_parts = 1;
+  size_t off_m = 0, off_l = 0, bytes = 0;
+};
+
+static size_t align256(size_t x) { return (x + 255) & ~static_cast<size_t>(255); }
+
+static int make_plan(int batch, int hq, int hkv, int d, int bs, int max_seq_len,
+                     int partition_tokens, Plan* plan) {
+  const int nblk_max = max_seq_len > 0 ? (max_seq_len + bs - 1) / bs : 1;
+  int pb;
+  if (partition_tokens > 0) {
+    if (partition_tokens % bs != 0)
+      return fail(PA_ERR_INVALID, "partition_tokens %d not a multiple of block_size %d",
+                  partition_tokens, bs);
+    pb = partition_tokens / bs;
+  } else {
+    // 512-token partitions; halve them while the grid would leave the SMs
+    // short of work (few, short requests).
+    pb = 512 / bs;
+    const int sms = sm_count() > 0 ? sm_count() : 148;
+    const long long pairs = static_cast<long long>(batch) * hkv;
+    while (pb > 4 && pairs * ((nblk_max + pb - 1) / pb) < 4ll * sms) pb /= 2;
+  }
+  pb = pb < 1 ? 1 : pb;
+  plan->part_blocks = pb;
+  plan->max_parts = (nblk_max + pb - 1) / pb;
+  if (plan->max_parts > 1) {
+    const size_t rows = static_cast<size_t>(batch) * hq * plan->max_parts;
+    plan->off_m = align256(rows * d * sizeof(float));
+    plan->off_l = plan->off_m + align256(rows * sizeof(float));
+    plan->bytes = plan->off_l + align256(rows * sizeof(float));
+  } else {
+    plan->off_m = plan->off_l = plan->bytes = 0;
+  }
+  return PA_OK;
+}
+
+static int check_shape(int batch, int hq, int hkv, int d, int bs, int max_seq_len) {
+  if (batch < 0 || hq <= 0 || hkv <= 0 || max_seq_len < 0)
+    return fail(PA_ERR_INVALID, "pa_decode: bad sizes (batch %d, heads %d/%d, max_seq_len %d)",
+                batch, hq, hkv, max_seq_len);
+  if (hq % hkv != 0)
+    return fail(PA_ERR_INVALID, "pa_decode: num_q_heads %d not a multiple of num_kv_heads %d", hq, hkv);
+  if (hq / hkv > kMaxGroup)
+    return fail(PA_ERR_UNSUPPORTED, "pa_decode: group size %d above %d", hq / hkv, kMaxGroup);
+  if (d != 64 && d != 128) return fail(PA_ERR_UNSUPPORTED, "pa_decode: head_dim %d not in {64,128}", d);
+  if (bs != 16 && bs != 32)
+    return fail(PA_ERR_UNSUPPORTED, "pa_decode: block_size %d not in {16,32}", bs);
+  if (batch > 65535 || hkv > 65535)
+    return fail(PA_ERR_UNSUPPORTED, "pa_decode: batch or num_kv_heads above 65535");
+  return PA_OK;
+}
+
+template <int D, int BS, int VAR, int G>
+static int launch_main(const CUtensorMap& map, const DecodeArgs& a, int batch, cudaStream_t st) {
+  using sm = Smem<D, BS, G>;
+  auto kern = paged_decode_kernel<D, BS, VAR, G>;
+  int rc = set_smem_attr(reinterpret_cast<const void*>(kern), sm::kDynamic);
+  if (rc != PA_OK) return rc;
+  dim3 grid(static_cast<unsigned>(a.max_parts), static_cast<unsigned>(a.num_kv_heads),
+            static_cast<unsigned>(batch));
+  kern<<<grid, kThreads, sm::kDynamic, st>>>(map, a);
+  PA_CUDA_TRY(cudaGetLastError());
+  return PA_OK;
+}
+
+template <int D, int BS>
+static int dispatch(const CUtensorMap& map, const DecodeArgs& a, int batch, int variant,
+                    cudaStream_t st) {
+  int rc;
+  if (variant == kMma) {
+    rc = launch_main<D, BS, kMma, 0>(map, a, batch, st);
+  } else {
+    switch (a.group) {
+      case 1: rc = launch_main<D, BS, kCudaCore, 1>(map, a, batch, st); break;
+      case 2: rc = launch_main<D, BS, kCudaCore, 2>(map, a, batch, st); break;
+      case 4: rc = launch_main<D, BS, kCudaCore, 4>(map, a, batch, st); break;
+      default:
+        return fail(PA_ERR_UNSUPPORTED, "pa_decode: CUDA-core variant has no group size %d", a.group);
+    }
+  }
+  if (rc != PA_OK) return rc;
+  if (a.max_parts > 1) {
+    const int warps = batch * a.num_q_heads;
+    paged_decode_reduce_kernel<D, BS><<<(warps + 3) / 4, 128, 0, st>>>(a, batch);
+    PA_CUDA_TRY(cudaGetLastError());
+  }
+  return PA_OK;
+}
+
+static int decode_impl(pa_bf16* out, const pa_bf16* q, const pa_bf16* kv_pool,
+                       const int32_t* block_tables, const int32_t* seq_lens, int batch, int hq,
+                       int hkv, int d, int bs, int num_blocks, int max_blocks, int max_seq_len,
+                       float scale, void* workspace, size_t ws_bytes, int variant,
+                       int partition_tokens, void* stream) {
+  int rc = check_shape(batch, hq, hkv, d, bs, max_seq_len);
+  if (rc != PA_OK) return rc;
+  if (num_blocks <= 0 || max_blocks <= 0)
+    return fail(PA_ERR_INVALID, "pa_decode: num_blocks and max_blocks_per_seq must be positive");
+  if (partition_tokens < 0) return fail(PA_ERR_INVALID, "pa_decode: negative partition_tokens");
+  if (!std::isfinite(scale)) return fail(PA_ERR_INVALID, "pa_decode: scale is not finite");
+  if (batch == 0) return PA_OK;
+  if (!out || !q || !kv_pool || !block_tables || !seq_lens)
+    return fail(PA_ERR_INVALID, "pa_decode: NULL pointer");
+  auto a16 = [](const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; };
+  if (!a16(out) || !a16(q) || !a16(kv_pool) || (reinterpret_cast<uintptr_t>(block_tables) & 3u) ||
+      (reinterpret_cast<uintptr_t>(seq_lens) & 3u))
+    return fail(PA_ERR_INVALID, "pa_decode: misaligned pointer");
+  const int group = hq / hkv;
+  if (variant == PA_DECODE_AUTO) variant = group >= 4 ? kMma : kCudaCore;
+  if (variant == kCudaCore && group != 1 && group != 2 && group != 4)
+    return fail(PA_ERR_UNSUPPORTED, "pa_decode: CUDA-core variant has no group size %d", group);
+  if (variant != kCudaCore && variant != kMma)
+    return fail(PA_ERR_INVALID, "pa_decode: unknown variant %d", variant);
+
+  Plan plan;
+  rc = make_plan(batch, hq, hkv, d, bs, max_seq_len, partition_tokens, &plan);
+  if (rc != PA_OK) return rc;
+  if (plan.bytes > 0) {
+    if (workspace == nullptr || ws_bytes < plan.bytes)
+      return fail(PA_ERR_INVALID, "pa_decode: workspace of %zu bytes needed, %zu given",
+                  plan.bytes, workspace ? ws_bytes : static_cast<size_t>(0));
+    if (reinterpret_cast<uintptr_t>(workspace) & 255u)
+      return fail(PA_ERR_INVALID, "pa_decode: workspace not 256-byte aligned");
+  }
+  int32_t* err = device_error_word();
+  if (err == nullptr) return PA_ERR_CUDA;
+
+  // TMA view of the pool: x = head dim, y = (kv head, row) of one K or V
+  // plane of a block, z = 2*block + (0 keys | 1 values).
+  alignas(64) CUtensorMap map;
+  const uint64_t dims[3] = {static_cast<uint64_t>(d), static_cast<uint64_t>(hkv) * bs,
+                            2ull * static_cast<uint64_t>(num_blocks)};
+  const uint64_t strides[2] = {static_cast<uint64_t>(d) * 2,
+                               static_cast<uint64_t>(hkv) * bs * d * 2};
+  const uint32_t box[3] = {64u, static_cast<uint32_t>(bs), 2u};
+  rc = encode_tensor_map(&map, 3, const_cast<pa_bf16*>(kv_pool), dims, strides, box, 1);
+  if (rc != PA_OK) return rc;
+
+  DecodeArgs a;
+  a.out = reinterpret_cast<__nv_bfloat16*>(out);
+  a.q = reinterpret_cast<const __nv_bfloat16*>(q);
+  a.block_tables = block_tables;
+  a.seq_lens = seq_lens;
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  a.part_o = plan.bytes ? reinterpret_cast<float*>(ws) : nullptr;
+  a.part_m = plan.bytes ? reinterpret_cast<float*>(ws + plan.off_m) : nullptr;
+  a.part_l = plan.bytes ? reinterpret_cast<float*>(ws + plan.off_l) : nullptr;
+  a.err = err;
+  a.num_q_heads = hq;
+  a.num_kv_heads = hkv;
+  a.group = group;
+  a.num_blocks = num_blocks;
+  a.max_blocks_per_seq = max_blocks;
+  a.part_blocks = plan.part_blocks;
+  a.max_parts = plan.max_parts;
+  a.scale_log2 = scale * 1.4426950408889634f;
+
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (d == 64 && bs == 16) return dispatch<64, 16>(map, a, batch, variant, st);
+  if (d == 64 && bs == 32) return dispatch<64, 32>(map, a, batch, variant, st);
+  if (d == 128 && bs == 16) return dispatch<128, 16>(map, a, batch, variant, st);
+  return dispatch<128, 32>(map, a, batch, variant, st);
+}
+
+}  // namespace pa
+
+extern "C" {
+
+int pa_decode_workspace_size_ex(int batch, int num_q_heads, int num_kv_heads, int head_dim,
+                                int block_size, int max_seq_len, int partition_tokens,
+                                size_t* bytes_out, int* num_partitions_out) {
+  using namespace pa;
+  if (bytes_out == nullptr) return fail(PA_ERR_INVALID, "pa_decode_workspace_size: NULL bytes_out");
+  int rc = check_shape(batch, num_q_heads, num_kv_heads, head_dim, block_size, max_seq_len);
+  if (rc != PA_OK) return rc;
+  if (partition_tokens < 0) return fail(PA_ERR_INVALID, "negative partition_tokens");
+  Plan plan;
+  rc = make_plan(batch, num_q_heads, num_kv_heads, head_dim, block_size, max_seq_len,
+                 partition_tokens, &plan);
+  if (rc != PA_OK) return rc;
+  *bytes_out = plan.bytes;
+  if (num_partitions_out) *num_partitions_out = plan.max_parts;
+  return PA_OK;
+}
+
+int pa_decode_workspace_size(int batch, int num_q_heads, int num_kv_heads, int head_dim,
+                             int block_size, int max_seq_len, size_t* bytes_out,
+                             int* num_partitions_out) {
+  return pa_decode_workspace_size_ex(batch, num_q_heads, num_kv_heads, head_dim, block_size,
+                                     max_seq_len, 0, bytes_out, num_partitions_out);
+}
+
+int pa_decode(pa_bf16* out, const pa_bf16* q, const pa_bf16* kv_pool, const int32_t* block_tables,
+              const int32_t* seq_lens, int batch, int num_q_heads, int num_kv_heads, int head_dim,
+              int block_size, int num_blocks, int max_blocks_per_seq, int max_seq_len, float scale,
+              void* workspace, size_t workspace_bytes, void* stream) {
+  return pa::decode_impl(out, q, kv_pool, block_tables, seq_lens, batch, num_q_heads,
+                         num_kv_heads, head_dim, block_size, num_blocks, max_blocks_per_seq,
+                         max_seq_len, scale, workspace, workspace_bytes, PA_DECODE_AUTO, 0, stream);
+}
+
+int pa_decode_ex(pa_bf16* out, const pa_bf16* q, const pa_bf16* kv_pool,
+                 const int32_t* block_tables, const int32_t* seq_lens, int batch, int num_q_heads,
+                 int num_kv_heads, int head_dim, int block_size, int num_blocks,
+                 int max_blocks_per_seq, int max_seq_len, float scale, void* workspace,
+                 size_t workspace_bytes, int variant, int partition_tokens, void* stream) {
+  return pa::decode_impl(out, q, kv_pool, block_tables, seq_lens, batch, num_q_heads,
+                         num_kv_heads, head_dim, block_size, num_blocks, max_blocks_per_seq,
+                         max_seq_len, scale, workspace, workspace_bytes, variant, partition_tokens,
+                         stream);
+}
+
+}  // extern "C"

@@ -1,0 +1,153 @@
+"""pa_decode parity with the fp64 oracle on small and ragged cases.
+
+Sizes span several partitions, stages and tiles with a ragged tail; every
+pool row that holds no token is NaN, so a kernel that reads past a request's
+end, or lets P=0 meet a NaN value, fails.  Tolerance (attention outputs vs
+fp64): max |err| <= 1e-2 and mean |err| <= 1e-3.
+"""
+
+import numpy as np
+import pytest
+import torch
+
+import paged_kv_cache_354_b200 as pk
+from oracle import paged_attention as opa
+from tests.gpu_helpers import (bf16_to_f64, build_tables, compare, default_scale, poison_unused,
+                               run_decode)
+import workloads
+
+pytestmark = pytest.mark.gpu
+
+VARIANTS = {"auto": pk.PA_DECODE_AUTO, "cuda_core": pk.PA_DECODE_CUDA_CORE, "mma": pk.PA_DECODE_MMA}
+
+
+def make_case(lens, hq, hkv, d, bs, seed, extra_blocks=4):
+    nb = sum(-(-int(n) // bs) for n in lens) + extra_blocks
+    rng = np.random.default_rng(seed)
+    order = rng.permutation(nb)
+    t_ref, l_ref, t_cpp, l_cpp, used = build_tables(lens, bs, nb, order)
+    pool = workloads.bf16_normal((nb, 2, hkv, bs, d), seed=seed)
+    poison_unused(pool, used)
+    q = workloads.bf16_normal((len(lens), hq, d), seed=seed + 1)
+    return q, pool, (t_ref, l_ref), (t_cpp, l_cpp)
+
+
+def check(lens, hq, hkv, d, bs, seed, variant="auto", partition_tokens=0, scale=None):
+    scale = default_scale(d) if scale is None else scale
+    q, pool, (t_ref, l_ref), (t_cpp, l_cpp) = make_case(lens, hq, hkv, d, bs, seed)
+    want = opa.decode(bf16_to_f64(q), bf16_to_f64(pool), t_ref, l_ref, scale)
+    out = run_decode(q.cuda(), pool.cuda(), t_cpp, l_cpp, scale, VARIANTS[variant], partition_tokens)
+    assert pk.pa_device_error() == 0
+    return compare(bf16_to_f64(out), want)
+
+
+RAGGED = [1, 15, 16, 17, 32, 53, 100, 257, 600]
+
+
+@pytest.mark.parametrize("d", [64, 128])
+@pytest.mark.parametrize("bs", [16, 32])
+@pytest.mark.parametrize("group", [1, 2, 4, 8])
+def test_auto_variant_ragged(d, bs, group):
+    hkv = 2
+    check(RAGGED, hkv * group, hkv, d, bs, seed=7 * d + bs + group)
+
+
+@pytest.mark.parametrize("variant,group", [("cuda_core", 1), ("cuda_core", 2), ("cuda_core", 4),
+                                           ("mma", 1), ("mma", 2), ("mma", 3), ("mma", 4), ("mma", 5),
+                                           ("mma", 8)])
+@pytest.mark.parametrize("d,bs", [(128, 16), (64, 32)])
+def test_each_variant(variant, group, d, bs):
+    check([5, 31, 33, 200, 480], 2 * group, 2, d, bs, seed=100 + group, variant=variant)
+
+
+@pytest.mark.parametrize("partition_blocks", [1, 2, 3, 8, 64])
+@pytest.mark.parametrize("variant", ["cuda_core", "mma"])
+def test_split_k_partitions(partition_blocks, variant):
+    """Many, few and a single partition agree with the oracle (split-K + LSE merge)."""
+    bs = 16
+    check([1, 16, 47, 300, 1000], 8, 2, 128, bs, seed=55, variant=variant,
+          partition_tokens=partition_blocks * bs)
+
+
+def test_split_k_consistency():
+    """P=1 and P>1 results agree to fp32-merge rounding, not just to the tolerance."""
+    lens = [700, 1024, 64]
+    q, pool, _, (t, l) = make_case(lens, 16, 4, 128, 16, seed=9)
+    q, pool = q.cuda(), pool.cuda()
+    one = run_decode(q, pool, t, l, 0.088, pk.PA_DECODE_MMA, partition_tokens=2048)
+    many = run_decode(q, pool, t, l, 0.088, pk.PA_DECODE_MMA, partition_tokens=64)
+    diff = (one.float() - many.float()).abs().max().item()
+    assert diff <= 2 ** -7, diff
+
+
+def test_cuda_core_and_mma_agree():
+    lens = [333, 90, 1500]
+    q, pool, _, (t, l) = make_case(lens, 8, 2, 128, 16, seed=10)
+    q, pool = q.cuda(), pool.cuda()
+    a = run_decode(q, pool, t, l, 0.1, pk.PA_DECODE_CUDA_CORE)
+    b = run_decode(q, pool, t, l, 0.1, pk.PA_DECODE_MMA)
+    assert (a.float() - b.float()).abs().max().item() <= 1e-2
+
+
+def test_length_one_returns_v():
+    """A request of length 1 attends to one token: out equals V exactly."""
+    lens = [1, 1, 1]
+    q, pool, (t_ref, _), (t, l) = make_case(lens, 8, 2, 128, 16, seed=11)
+    for variant in (pk.PA_DECODE_CUDA_CORE, pk.PA_DECODE_MMA):
+        out = run_decode(q.cuda(), pool.cuda(), t, l, 0.3, variant).cpu()
+        for b in range(3):
+            for j in range(8):
+                assert torch.equal(out[b, j], pool[t_ref[b, 0], 1, j // 4, 0])
+
+
+def test_zero_length_request():
+    lens = [0, 40, 0, 7]
+    q, pool, (t_ref, l_ref), (t, l) = make_case(lens, 4, 4, 64, 16, seed=12)
+    out = run_decode(q.cuda(), pool.cuda(), t, l, 0.125).cpu()
+    assert torch.count_nonzero(out[0]) == 0 and torch.count_nonzero(out[2]) == 0
+    want = opa.decode(bf16_to_f64(q), bf16_to_f64(pool), t_ref, l_ref, 0.125)
+    compare(bf16_to_f64(out), want)
+
+
+def test_large_logits():
+    """A large scale makes the softmax nearly one-hot; the online max must hold."""
+    check([77, 500], 8, 2, 128, 16, seed=13, scale=4.0)
+    check([77, 500], 4, 4, 64, 16, seed=14, scale=4.0)
+
+
+def test_tiny_workload():
+    """The tiny workload end to end: lengths U[1,64], one appended token."""
+    p = workloads.plan("tiny")
+    s = p.shape
+    lens = [int(n) + 1 for n in p.seq_lens]
+    check(lens, s.num_q_heads, s.num_kv_heads, s.head_dim, s.block_size, seed=workloads.seed_of("tiny"))
+
+
+def test_device_checks_flag_bad_inputs():
+    """Bad block ids / lengths are flagged, skipped or clamped; nothing faults."""
+    lens = [40, 40]
+    q, pool, _, (t, l) = make_case(lens, 4, 2, 128, 16, seed=15)
+    q, pool = q.cuda(), pool.cuda()
+    pk.pa_device_error(clear=True)
+    bad = t.copy()
+    bad[0, 1] = pool.shape[0] + 5
+    run_decode(q, pool, bad, l, 0.1)
+    assert pk.pa_device_error() & pk.PA_DEVERR_BLOCK_ID
+    long_lens = l.copy()
+    long_lens[1] = t.shape[1] * 16 + 9  # beyond the table row
+    ws = torch.empty(1 << 20, dtype=torch.uint8, device="cuda")
+    out = torch.empty_like(q)
+    pk.pa_decode(out, q, pool, torch.as_tensor(t, device="cuda"), torch.as_tensor(long_lens, device="cuda"),
+                 int(long_lens.max()), 0.1, workspace=ws)
+    torch.cuda.synchronize()
+    assert pk.pa_device_error() & pk.PA_DEVERR_SEQ_LEN
+    assert pk.pa_device_error() == 0  # cleared by the previous read
+
+
+def test_wait_timeout_is_reported():
+    pk.pa_device_error(clear=True)
+    pk.pa_selftest_wait_timeout(20_000_000)  # 20 ms
+    torch.cuda.synchronize()
+    assert pk.pa_device_error() == pk.PA_DEVERR_WAIT_TIMEOUT
+    # the context is still usable
+    check([20], 4, 4, 64, 16, seed=16)
