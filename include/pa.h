@@ -188,6 +188,37 @@ int pa_decode_ex(pa_bf16* out, const pa_bf16* q, const pa_bf16* kv_pool,
                  void* workspace, size_t workspace_bytes, int variant,
                  int partition_tokens, void* stream);
 
+/* --------------------------------------------------------------------------
+ * pa_decode_noalloc -- pa_decode for callers that cannot allocate device
+ * memory.  (No counterpart on the pages: this is a packaging choice.)
+ *
+ * Some callers have no way to hand the library a workspace: a plugin
+ * running inside a host program that owns the whole GPU memory budget and
+ * forbids its own cudaMalloc calls, or a latency-critical decode loop where
+ * cudaMalloc's implicit device synchronisation is not acceptable.  This
+ * entry point takes the same arguments as pa_decode minus the workspace and
+ * keeps the split-K partials in a fixed array compiled into the library
+ * (PA_NOALLOC_SCRATCH_BYTES on every GPU that loads the library, held until
+ * the process exits).  It calls no cudaMalloc/cudaFree and no allocating
+ * library routine.
+ *  - A call whose split-K scratch (pa_decode_workspace_size for the same
+ *    arguments) exceeds PA_NOALLOC_SCRATCH_BYTES returns PA_ERR_UNSUPPORTED
+ *    before launching anything; use pa_decode with a caller workspace.
+ *  - The first call on each device looks up the array's device address
+ *    (cudaGetSymbolAddress) with that device current; make that first call
+ *    before any stream capture.
+ *  - Every call on a device shares the one array and it keeps the last
+ *    call's contents; nothing in it needs to start at zero.  Calls that can
+ *    overlap on the GPU (different streams without ordering) race on it.
+ * ------------------------------------------------------------------------ */
+#define PA_NOALLOC_SCRATCH_BYTES (16u * 1024u * 1024u)
+
+int pa_decode_noalloc(pa_bf16* out, const pa_bf16* q, const pa_bf16* kv_pool,
+                      const int32_t* block_tables, const int32_t* seq_lens, int batch,
+                      int num_q_heads, int num_kv_heads, int head_dim, int block_size,
+                      int num_blocks, int max_blocks_per_seq, int max_seq_len, float scale,
+                      void* stream);
+
 /* Self-test of the bounded pipeline wait used by the kernels: one CTA waits
  * on a barrier phase that nothing completes, for at most limit_ns, then
  * returns.  Expect PA_DEVERR_WAIT_TIMEOUT in pa_device_error() afterwards.

@@ -5,7 +5,7 @@ here has the C entry point's name and only turns tensors into pointers and
 the current CUDA stream into a handle.  All work runs in the library's
 kernels; there is no Python or CPU fallback.  Importing this package raises
 if ``libpa.so`` is missing (build it with
-``python -m paged_kv_cache_354_b200._build``).
+``python paged_kv_cache_354_b200/_build.py``).
 
 bf16 tensors are ``torch.bfloat16``; shapes follow ``include/pa.h``:
     kv_pool      [num_blocks, 2, num_kv_heads, block_size, head_dim]
@@ -58,6 +58,7 @@ _SIGNATURES = {
     "pa_decode": (_I, [_P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _I, _I, _c.c_float, _P, _SZ, _P]),
     "pa_decode_ex": (_I, [_P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _I, _I, _c.c_float, _P, _SZ,
                           _I, _I, _P]),
+    "pa_decode_noalloc": (_I, [_P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _I, _I, _c.c_float, _P]),
     "pa_selftest_wait_timeout": (_I, [_I64, _P]),
     "pa_alloc_create": (_I, [_I, _I, _P, _P]),
     "pa_alloc_destroy": (_I, [_P]),
@@ -78,7 +79,7 @@ _SIGNATURES = {
 def _load():
     if not os.path.exists(_LIB_PATH):
         raise ImportError(
-            f"{_LIB_PATH} is missing: build it with `python -m paged_kv_cache_354_b200._build`"
+            f"{_LIB_PATH} is missing: build it with `python paged_kv_cache_354_b200/_build.py`"
         )
     lib = ctypes.CDLL(_LIB_PATH)
     for name, (res, args) in _SIGNATURES.items():
@@ -205,6 +206,30 @@ def pa_decode(out, q, kv_pool, block_tables, seq_lens, max_seq_len, scale, works
     _check(lib.pa_decode_ex(_ptr(out), _ptr(q), _ptr(kv_pool), _ptr(block_tables), _ptr(seq_lens), b, hq,
                             hkv, d, bs, nb, block_tables.shape[1], int(max_seq_len), float(scale), ws_ptr,
                             ws_bytes, int(variant), int(partition_tokens), _stream(stream)), "pa_decode")
+
+
+PA_NOALLOC_SCRATCH_BYTES = 16 * 1024 * 1024
+
+
+def pa_decode_noalloc(out, q, kv_pool, block_tables, seq_lens, max_seq_len, scale, stream=None):
+    """pa_decode without a workspace argument, for callers that cannot
+    allocate device memory: the split-K partials live in a fixed array of
+    PA_NOALLOC_SCRATCH_BYTES inside the library (shared by all calls on a
+    device; calls that overlap on the GPU race on it)."""
+    import torch
+
+    _require(out, torch.bfloat16, "out")
+    _require(q, torch.bfloat16, "q")
+    _require(kv_pool, torch.bfloat16, "kv_pool")
+    _require(block_tables, torch.int32, "block_tables")
+    _require(seq_lens, torch.int32, "seq_lens")
+    nb, two, hkv, bs, d = kv_pool.shape
+    b, hq, dq = q.shape
+    if out.shape != q.shape or dq != d or block_tables.shape[0] != b or seq_lens.shape != (b,):
+        raise ValueError("pa_decode_noalloc: shape mismatch")
+    _check(lib.pa_decode_noalloc(_ptr(out), _ptr(q), _ptr(kv_pool), _ptr(block_tables), _ptr(seq_lens), b,
+                                 hq, hkv, d, bs, nb, block_tables.shape[1], int(max_seq_len), float(scale),
+                                 _stream(stream)), "pa_decode_noalloc")
 
 
 def pa_selftest_wait_timeout(limit_ns, stream=None):
