@@ -1,9 +1,11 @@
 """Build libpa.so in-tree with nvcc for sm_100a.
 
-    python -m paged_kv_cache_354_b200._build [--force] [--verbose]
+    python paged_kv_cache_354_b200/_build.py [--force] [--verbose]
 
 Objects go to ``_build/`` at the repository root; the shared library is
-written next to this file, where the binding loads it.
+written next to this file, where the binding loads it.  Run it as a script
+(or load it by path): importing the package first would load the library
+this script is about to rebuild.
 """
 
 import argparse
