@@ -120,7 +120,12 @@ def decode_bytes(lens, hq, hkv, d, bs):
     return kv + qo + tables, kv
 
 
-def build_cache(name, steps_total, rank, device):
+def build_cache(name, steps_total, rank, device, prefill=True):
+    """Pool (seeded bf16 N(0,1)), allocator state and request ids of a workload.
+
+    With ``prefill`` the beam workload's 256 divergent tokens per beam are
+    appended (copy-on-write + cache write) before the decode loop starts.
+    """
     import torch
 
     from paged_kv_cache_354_b200.engine import PagedDecodeCache
@@ -132,21 +137,31 @@ def build_cache(name, steps_total, rank, device):
     batch = len(lens0) * (p.beams or 1)
     cache = PagedDecodeCache(p.num_blocks, s.num_q_heads, s.num_kv_heads, s.head_dim, s.block_size,
                              batch, max_len, initial_order=p.initial_order, device=device)
-    # pool content: bf16 N(0,1) from a seeded device generator (rank-distinct)
     gen = torch.Generator(device=device)
     gen.manual_seed(workloads.seed_of(name) * 1000 + rank)
     cache.pool.copy_(torch.randn(cache.pool.shape, generator=gen, device=device,
                                  dtype=torch.float32).to(torch.bfloat16))
     ids = workloads.populate(cache.alloc, p)
-    if p.name == "beam":  # the 256 divergent tokens per beam go in before the decode loop
-        slots, pairs = cache.alloc.append_batch(ids, p.append_tokens, as_numpy=True)
-        k = torch.randn((len(slots), s.num_kv_heads, s.head_dim), generator=gen, device=device).bfloat16()
-        v = torch.randn((len(slots), s.num_kv_heads, s.head_dim), generator=gen, device=device).bfloat16()
-        from paged_kv_cache_354_b200 import pa_copy_blocks, pa_reshape_and_cache
-
-        pa_copy_blocks(cache.pool, torch.as_tensor(pairs, device=device))
-        pa_reshape_and_cache(k, v, cache.pool, torch.as_tensor(slots, device=device))
+    if prefill and p.name == "beam":
+        beam_prefill(p, cache, ids, gen, device)
     return p, cache, ids, gen
+
+
+def beam_prefill(p, cache, ids, gen, device):
+    """Append each beam's divergent tokens: allocator, copy_blocks, cache write.
+
+    Returns (slots, pairs, k, v) as used, for an independent replay."""
+    import torch
+
+    from paged_kv_cache_354_b200 import pa_copy_blocks, pa_reshape_and_cache
+
+    s = p.shape
+    slots, pairs = cache.alloc.append_batch(ids, p.append_tokens, as_numpy=True)
+    k = torch.randn((len(slots), s.num_kv_heads, s.head_dim), generator=gen, device=device).bfloat16()
+    v = torch.randn((len(slots), s.num_kv_heads, s.head_dim), generator=gen, device=device).bfloat16()
+    pa_copy_blocks(cache.pool, torch.as_tensor(pairs, device=device))
+    pa_reshape_and_cache(k, v, cache.pool, torch.as_tensor(slots, device=device))
+    return slots, pairs, k, v
 
 
 def make_inputs(cache, batch, gen, device):
@@ -164,6 +179,22 @@ def make_inputs(cache, batch, gen, device):
 # --------------------------------------------------------------------------
 # the GPU arm
 # --------------------------------------------------------------------------
+def combine_ranks(times_ms, totals, device, world):
+    """Whole-job figures: the max of every rank's times, the sum of their work.
+
+    Works on any process group backend (NCCL on the GPUs, gloo in the CPU
+    tests); with one rank it returns the inputs."""
+    import torch
+    import torch.distributed as dist
+
+    t = torch.tensor(list(times_ms), device=device, dtype=torch.float64)
+    w = torch.tensor(list(totals), device=device, dtype=torch.float64)
+    if world > 1:
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        dist.all_reduce(w, op=dist.ReduceOp.SUM)
+    return tuple(t.tolist()) + tuple(w.tolist())
+
+
 def run_gpu(args):
     import torch
     import torch.distributed as dist
@@ -229,52 +260,52 @@ def run_gpu(args):
     kv_timed = sum(kv for _, kv in step_bytes[W:])
 
     # ---- end-to-end arm: host allocator + pinned H2D + kernels + D2H per step
+    # (the device part of the step is a CUDA graph recorded once)
     h_q = [t.cpu().pin_memory() for t in qs]
     h_k = [t.cpu().pin_memory() for t in ks]
     h_v = [t.cpu().pin_memory() for t in vs]
     d_q, d_k, d_v = torch.empty_like(qs[0]), torch.empty_like(ks[0]), torch.empty_like(vs[0])
     h_out = torch.empty(out.shape, dtype=out.dtype).pin_memory()
-    e2e_bytes, e2e_h2d = 0, 0
+    e2e_lens = []
 
     def e2e_step(i):
-        nonlocal e2e_bytes, e2e_h2d
         j = i % INPUT_SETS
-        slots, pairs, tables, lens = cache.plan_append(ids)
-        npairs = cache.stage(slots, pairs, tables, lens)
+        npairs = cache.host_step(ids)
+        cache.upload()
         d_q.copy_(h_q[j], non_blocking=True)
         d_k.copy_(h_k[j], non_blocking=True)
         d_v.copy_(h_v[j], non_blocking=True)
-        cache.run(d_q, d_k, d_v, out, cache.d_slots[:batch], cache.d_tables[:batch], cache.d_lens[:batch],
-                  cache.d_pairs[:npairs])
+        cache.replay(npairs)
         h_out.copy_(out, non_blocking=True)
-        torch.cuda.current_stream().synchronize()
-        return decode_bytes(lens, cache.hq, cache.hkv, cache.d, cache.bs)[0], (
-            slots.nbytes + tables.nbytes + lens.nbytes + 8 * npairs + h_q[j].nbytes + 2 * h_k[j].nbytes)
+        stream.synchronize()
+        e2e_lens.append(cache.h_lens[:batch].numpy().copy())
 
+    cache.host_step(ids)  # one eager step, then record the graph on its staged metadata
+    cache.upload()
+    d_q.copy_(h_q[0])
+    d_k.copy_(h_k[0])
+    d_v.copy_(h_v[0])
+    cache.capture(d_q, d_k, d_v, out)
     for i in range(W):
         e2e_step(i)
     torch.cuda.synchronize()
     if world > 1:
         dist.barrier()
+    e2e_lens.clear()
     e_start, e_end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     e_start.record(stream)
     for i in range(K):
-        nb, h2d = e2e_step(W + i)
-        e2e_bytes += nb
-        e2e_h2d += h2d
+        e2e_step(W + i)
     e_end.record(stream)
     torch.cuda.synchronize()
     e2e_ms = e_start.elapsed_time(e_end)
+    e2e_bytes = sum(decode_bytes(ln, cache.hq, cache.hkv, cache.d, cache.bs)[0] for ln in e2e_lens)
+    e2e_h2d = K * (cache.meta_bytes + h_q[0].nbytes + h_k[0].nbytes + h_v[0].nbytes)
     dev_err = pa_device_error()
 
-    # ---- max over ranks
-    times = torch.tensor([dev_ms, e2e_ms, float(np.mean(decode_ms))], device=device, dtype=torch.float64)
-    totals = torch.tensor([bytes_timed, e2e_bytes, kv_timed], device=device, dtype=torch.float64)
-    if world > 1:
-        dist.all_reduce(times, op=dist.ReduceOp.MAX)
-        dist.all_reduce(totals, op=dist.ReduceOp.SUM)
-    dev_ms, e2e_ms, decode_avg_ms = times.tolist()
-    bytes_all, e2e_bytes_all, kv_all = totals.tolist()
+    # ---- max over ranks (times), sum over ranks (work)
+    dev_ms, e2e_ms, decode_avg_ms, bytes_all, e2e_bytes_all, kv_all = combine_ranks(
+        [dev_ms, e2e_ms, float(np.mean(decode_ms))], [bytes_timed, e2e_bytes, kv_timed], device, world)
 
     if rank == 0:
         peaks = load_peaks()
@@ -299,7 +330,9 @@ def run_gpu(args):
                 "batch": batch, "num_q_heads": cache.hq, "num_kv_heads": cache.hkv, "head_dim": cache.d,
                 "block_size": cache.bs, "num_blocks": cache.num_blocks,
                 "mean_seq_len": round(float(np.mean(plans[W][3])), 1),
-                "split_k_partitions": cache.num_partitions,
+                "decode_schedule": (f"balanced persistent: {cache.num_partitions} CTAs"
+                                    if cache.partition_tokens == 0 else
+                                    f"per-partition grid: {cache.num_partitions} partitions"),
                 "l2": f"inputs larger than L2: KV read per step {step_bytes[W][1] / 1e6:.0f} MB > 126 MB",
                 "parallelism": f"dp{world} (independent batches, no collective)",
             },
@@ -319,6 +352,8 @@ def run_gpu(args):
                 "value": round(e2e_bytes_all / (e2e_ms * 1e-3) / 1e9, 2),
                 "unit": "GB/s",
                 "h2d_bytes_per_step": int(e2e_h2d / K),
+                "path": "C++ allocator into pinned staging, 4 H2D copies, CUDA-graph replay of "
+                        "cache write + decode + merge, D2H of the output, sync",
                 "d2h_bytes_per_step": int(h_out.nbytes),
                 "ms_per_step": round(e2e_ms / K, 5),
             },

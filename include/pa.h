@@ -151,10 +151,19 @@ int pa_copy_blocks(pa_bf16* kv_pool, const int32_t* block_pairs, int num_pairs,
  * workspace    : device scratch of at least pa_decode_workspace_size() bytes
  *                (fp32 partial outputs and log-sum-exp terms of the
  *                sequence partitions), 256-byte aligned; its contents need
- *                no initialisation.  May be NULL when that size is 0.
+ *                no initialisation.
+ * Schedule: batches of up to 4096 requests use a balanced persistent
+ * schedule -- two CTAs per SM, each taking an equal contiguous share of all
+ * (request, KV head, block) units -- followed by a log-sum-exp merge of the
+ * (request, head) pairs cut between CTAs.  Larger batches use one CTA per
+ * (request, KV head, 512-token partition) and the same kind of merge.
  * Supported: head_dim in {64, 128}; block_size in {16, 32}; num_q_heads a
  * multiple of num_kv_heads with group size 1..8.  Others: PA_ERR_UNSUPPORTED.
+ * Launches: two kernels (decode + merge); the per-partition schedule skips
+ * the merge when no request spans two partitions.
  * ------------------------------------------------------------------------ */
+/* *num_partitions_out: CTAs of the balanced schedule, or sequence
+ * partitions of the per-partition schedule (merge launched when > 1). */
 int pa_decode_workspace_size(int batch, int num_q_heads, int num_kv_heads, int head_dim,
                              int block_size, int max_seq_len, size_t* bytes_out,
                              int* num_partitions_out);
@@ -174,9 +183,11 @@ typedef enum pa_decode_variant {
 
 /* pa_decode with explicit choices, for measurement and tests.
  * variant          : pa_decode_variant.
- * partition_tokens : tokens per split-K partition (a multiple of block_size),
- *                    or 0 for the built-in heuristic.  The workspace must be
- *                    sized with pa_decode_workspace_size_ex for the same value. */
+ * partition_tokens : 0 = the built-in schedule (see pa_decode); > 0 = one
+ *                    CTA per (request, KV head, partition of this many
+ *                    tokens, a multiple of block_size).  The workspace must
+ *                    be sized with pa_decode_workspace_size_ex for the same
+ *                    value. */
 int pa_decode_workspace_size_ex(int batch, int num_q_heads, int num_kv_heads, int head_dim,
                                 int block_size, int max_seq_len, int partition_tokens,
                                 size_t* bytes_out, int* num_partitions_out);

@@ -14,6 +14,8 @@ __global__ void __launch_bounds__(256) reshape_and_cache_kernel(
     const uint4* __restrict__ key, const uint4* __restrict__ value, uint4* __restrict__ pool,
     const int64_t* __restrict__ slot_mapping, int64_t total, int num_kv_heads, int block_size,
     int chunks, int64_t num_slots, int32_t* err) {
+  pdl_trigger();
+  pdl_wait();
   const int64_t idx = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
   if (idx >= total) return;
   const int chunk = static_cast<int>(idx % chunks);
@@ -43,6 +45,8 @@ constexpr int kCopyUnroll = 4;
 __global__ void __launch_bounds__(kCopyThreads) copy_blocks_kernel(
     uint4* __restrict__ pool, const int32_t* __restrict__ pairs, int num_blocks,
     int64_t vecs_per_block, int32_t* err) {
+  pdl_trigger();
+  pdl_wait();
   const int src = __ldg(pairs + 2 * blockIdx.x);
   const int dst = __ldg(pairs + 2 * blockIdx.x + 1);
   if (static_cast<unsigned>(src) >= static_cast<unsigned>(num_blocks) ||
@@ -93,11 +97,11 @@ int pa_reshape_and_cache(const pa_bf16* key, const pa_bf16* value, pa_bf16* kv_p
   const int64_t total = static_cast<int64_t>(num_tokens) * num_kv_heads * 2 * chunks;
   const int64_t grid = (total + 255) / 256;
   if (grid > 0x7fffffffll) return fail(PA_ERR_INVALID, "pa_reshape_and_cache: too many tokens");
-  reshape_and_cache_kernel<<<static_cast<unsigned>(grid), 256, 0, static_cast<cudaStream_t>(stream)>>>(
-      reinterpret_cast<const uint4*>(key), reinterpret_cast<const uint4*>(value),
-      reinterpret_cast<uint4*>(kv_pool), slot_mapping, total, num_kv_heads, block_size, chunks,
-      static_cast<int64_t>(num_blocks) * block_size, err);
-  PA_CUDA_TRY(cudaGetLastError());
+  PA_CUDA_TRY(launch_pdl(reshape_and_cache_kernel, dim3(static_cast<unsigned>(grid)), dim3(256), 0,
+                         static_cast<cudaStream_t>(stream), reinterpret_cast<const uint4*>(key),
+                         reinterpret_cast<const uint4*>(value), reinterpret_cast<uint4*>(kv_pool),
+                         slot_mapping, total, num_kv_heads, block_size, chunks,
+                         static_cast<int64_t>(num_blocks) * block_size, err));
   return PA_OK;
 }
 
@@ -120,9 +124,9 @@ int pa_copy_blocks(pa_bf16* kv_pool, const int32_t* block_pairs, int num_pairs, 
   const int64_t slices = (vecs + per_cta - 1) / per_cta;
   if (slices > 65535) return fail(PA_ERR_UNSUPPORTED, "pa_copy_blocks: block too large");
   dim3 grid(static_cast<unsigned>(num_pairs), static_cast<unsigned>(slices));
-  copy_blocks_kernel<<<grid, kCopyThreads, 0, static_cast<cudaStream_t>(stream)>>>(
-      reinterpret_cast<uint4*>(kv_pool), block_pairs, num_blocks, vecs, err);
-  PA_CUDA_TRY(cudaGetLastError());
+  PA_CUDA_TRY(launch_pdl(copy_blocks_kernel, grid, dim3(kCopyThreads), 0,
+                         static_cast<cudaStream_t>(stream), reinterpret_cast<uint4*>(kv_pool),
+                         block_pairs, num_blocks, vecs, err));
   return PA_OK;
 }
 

@@ -53,8 +53,10 @@ struct Geo {
   static constexpr int kStages = (kStageBytes <= 8192) ? 8 : 4;
   static constexpr int kStageSmem = kStages * kStageBytes;
   static_assert(kStages % kConsumerWarps == 0, "stage s must always go to warp s % warps");
-  // epilogue scratch aliased on the stage ring
-  static constexpr int kEpiO = kConsumerWarps * kMaxGroup * D * 4;
+  // epilogue scratch aliased on the stage ring; head rows padded by 4
+  // floats so the tensor-core store pattern hits 32 distinct banks
+  static constexpr int kOStride = D + 4;
+  static constexpr int kEpiO = kConsumerWarps * kMaxGroup * kOStride * 4;
   static constexpr int kEpiBytes = kEpiO + 2 * kConsumerWarps * kMaxGroup * 4;
   static_assert(kEpiBytes <= kStageSmem, "epilogue scratch must fit in the stage ring");
 };
@@ -85,6 +87,7 @@ struct DecodeArgs {
   int num_blocks, max_blocks_per_seq;
   int part_blocks, max_parts;
   float scale_log2;  // scale * log2(e)
+  int* stream_prefix;  // balanced schedule: per-request block-count prefix sums [B+1]
 };
 
 // Tokens of request b the kernels attend over, after the device-side checks
@@ -208,7 +211,7 @@ struct MmaConsumer {
   }
 
   // Write this warp's unnormalised O, running max and sum to the epilogue
-  // scratch: o_s[head][dim], m_s[head], l_s[head].
+  // scratch: o_s[head][dim] (row stride kOStride), m_s[head], l_s[head].
   __device__ __forceinline__ void store(float* o_s, float* m_s, float* l_s, int lane) {
 #pragma unroll
     for (int off = 4; off < 32; off <<= 1) {
@@ -219,10 +222,11 @@ struct MmaConsumer {
 #pragma unroll
     for (int dt = 0; dt < kDT; ++dt) {
       const int d = 16 * dt + (lane >> 2);
-      o_s[h0 * D + d] = o[dt][0];
-      o_s[(h0 + 1) * D + d] = o[dt][1];
-      o_s[h0 * D + d + 8] = o[dt][2];
-      o_s[(h0 + 1) * D + d + 8] = o[dt][3];
+      constexpr int S = geo::kOStride;
+      o_s[h0 * S + d] = o[dt][0];
+      o_s[(h0 + 1) * S + d] = o[dt][1];
+      o_s[h0 * S + d + 8] = o[dt][2];
+      o_s[(h0 + 1) * S + d + 8] = o[dt][3];
     }
     if (lane < 4) {
       m_s[h0] = m0;
@@ -382,7 +386,7 @@ struct CudaCoreConsumer {
 #pragma unroll
       for (int off = 4; off < 32; off <<= 1) lj += __shfl_xor_sync(kFull, lj, off);
 #pragma unroll
-      for (int e = 0; e < kOD; ++e) o_s[j * D + lane * kOD + e] = o[j][e];
+      for (int e = 0; e < kOD; ++e) o_s[j * geo::kOStride + lane * kOD + e] = o[j][e];
       if (lane == 0) {
         m_s[j] = m[j];
         l_s[j] = lj;
@@ -390,6 +394,39 @@ struct CudaCoreConsumer {
     }
   }
 };
+
+// --------------------------------------------------------------------------
+// One consumer warp's work on one staged block (shared by both schedules).
+// --------------------------------------------------------------------------
+template <int D, int BS, int VAR, int G>
+__device__ __forceinline__ void consume_block(MmaConsumer<D, BS>& mc,
+                                              CudaCoreConsumer<D, BS, (G > 0 ? G : 1)>& cc,
+                                              uint32_t sb, float* pbuf, int valid, float scale_log2,
+                                              int lane) {
+  using geo = Geo<D, BS>;
+  if constexpr (VAR == kMma) {
+    if (valid < BS) {
+      // rows past the end may hold anything, even NaN: zero their V so that
+      // P = 0 there contributes exactly 0
+      const int rows = BS - valid;
+      for (int t = lane; t < rows * geo::kRegions * 8; t += 32) {
+        const int r = valid + t / (geo::kRegions * 8);
+        const int x = (t / 8) % geo::kRegions;
+        const int ch = t % 8;
+        asm volatile("st.shared.v4.u32 [%0], {%1, %1, %1, %1};" ::"r"(
+                         sb + x * geo::kRegionBytes + (BS + r) * 128 + ch * 16),
+                     "r"(0u)
+                     : "memory");
+      }
+      // order these generic writes before the next TMA refill of the stage
+      fence_proxy_async_smem();
+      __syncwarp();
+    }
+    mc.step(sb, valid, scale_log2, lane);
+  } else {
+    cc.step(sb, pbuf, valid, scale_log2, lane);
+  }
+}
 
 // --------------------------------------------------------------------------
 // The decode kernel.  grid = (max_parts, num_kv_heads, batch).
@@ -412,6 +449,8 @@ __global__ void __launch_bounds__(kThreads, (VAR == kMma || G <= 2) ? 3 : 2)
   const int lane = threadIdx.x & 31;
   const int g = a.group;
 
+  pdl_trigger();
+  pdl_wait();  // every global access below comes after the previous grid
   const int len = effective_len(__ldg(a.seq_lens + b), BS, a, part == 0 && threadIdx.x == 0);
   const int nblk = (len + BS - 1) / BS;
   const int nparts = (nblk + a.part_blocks - 1) / a.part_blocks;
@@ -506,35 +545,14 @@ __global__ void __launch_bounds__(kThreads, (VAR == kMma || G <= 2) ? 3 : 2)
       }
       const uint32_t sb = sbase + s * geo::kStageBytes;
       const int valid = (blk0 + i == nblk - 1) ? last_valid : BS;
-      if constexpr (VAR == kMma) {
-        if (valid < BS) {
-          // rows past the end may hold anything, even NaN: zero their V so
-          // that P = 0 there contributes exactly 0
-          const int rows = BS - valid;
-          for (int t = lane; t < rows * geo::kRegions * 8; t += 32) {
-            const int r = valid + t / (geo::kRegions * 8);
-            const int x = (t / 8) % geo::kRegions;
-            const int ch = t % 8;
-            asm volatile("st.shared.v4.u32 [%0], {%1, %1, %1, %1};" ::"r"(
-                             sb + x * geo::kRegionBytes + (BS + r) * 128 + ch * 16),
-                         "r"(0u)
-                         : "memory");
-          }
-          // order these generic writes before the next TMA refill of the stage
-          fence_proxy_async_smem();
-          __syncwarp();
-        }
-        mc.step(sb, valid, a.scale_log2, lane);
-      } else {
-        cc.step(sb, pbuf, valid, a.scale_log2, lane);
-      }
+      consume_block<D, BS, VAR, G>(mc, cc, sb, pbuf, valid, a.scale_log2, lane);
       __syncwarp();
       if (lane == 0) mbar_arrive(bar_empty + 8 * s);
     }
   }
   __syncthreads();  // (A) the stage ring is idle; it becomes epilogue scratch
   if (warp < kConsumerWarps && *abort_flag == 0) {
-    float* o_s = reinterpret_cast<float*>(smem) + warp * kMaxGroup * D;
+    float* o_s = reinterpret_cast<float*>(smem) + warp * kMaxGroup * geo::kOStride;
     float* m_s = reinterpret_cast<float*>(smem + geo::kEpiO) + warp * kMaxGroup;
     float* l_s = m_s + kConsumerWarps * kMaxGroup;
     if constexpr (VAR == kMma) mc.store(o_s, m_s, l_s, lane);
@@ -582,7 +600,7 @@ __global__ void __launch_bounds__(kThreads, (VAR == kMma || G <= 2) ? 3 : 2)
 #pragma unroll
     for (int w = 0; w < kConsumerWarps; ++w) {
       const float f = fw[w * kMaxGroup + j];
-      const float* ow = o_all + (w * kMaxGroup + j) * D + d;
+      const float* ow = o_all + (w * kMaxGroup + j) * geo::kOStride + d;
       v0 = fmaf(f, ow[0], v0);
       v1 = fmaf(f, ow[1], v1);
     }
@@ -601,13 +619,447 @@ __global__ void __launch_bounds__(kThreads, (VAR == kMma || G <= 2) ? 3 : 2)
 }
 
 // --------------------------------------------------------------------------
+// Balanced ("stream") schedule.
+//
+// Work units are (request b, KV head h, block k) in that order; there are
+// U = Hkv * sum_b ceil(L_b / bs) of them.  A fixed grid of C CTAs (two per
+// SM) gives CTA c the contiguous units [floor(U c / C), floor(U (c+1) / C)),
+// so every CTA streams the same number of blocks and the whole batch runs in
+// one wave with no tail.  A CTA walks its range as segments of constant
+// (b, h): a segment that covers all of its (b, h) writes the bf16 output; a
+// segment cut by the CTA's range start or end (only the first and the last
+// can be) writes an fp32 partial into slot 0 (first) or 1 (last) of the CTA,
+// merged afterwards by paged_decode_stream_merge_kernel.
+// --------------------------------------------------------------------------
+constexpr int kStreamCtasPerSm = 2;
+constexpr int kStreamMaxBatch = 4096;  // the prefix table lives in shared memory
+
+template <int D, int BS, int G>
+struct StreamSmem {
+  using geo = Geo<D, BS>;
+  static constexpr int kBar = geo::kStageSmem;                   // full[S], empty[S]
+  static constexpr int kMisc = kBar + 16 * geo::kStages;         // last_round[S], abort
+  static constexpr int kScan = (kMisc + 4 * geo::kStages + 4 + 15) & ~15;  // scan scratch
+  static constexpr int kPbuf = kScan + (kThreads + 4) * 4;       // CUDA-core p tiles
+  static constexpr int kPbufBytes = kConsumerWarps * BS * (G > 0 ? G : 1) * 4;
+  static constexpr int kEpi = (kPbuf + kPbufBytes + 15) & ~15;   // per-warp O, m, l
+  static constexpr int kPrefix = kEpi + geo::kEpiBytes;          // int32 [batch + 1]
+  static constexpr int dynamic_bytes(int batch) { return kPrefix + 4 * (batch + 1) + 1024; }
+};
+
+// First unit of the CTA range that contains unit u: the largest c with
+// floor(total * c / ctas) <= u.
+__device__ __forceinline__ long long stream_begin(long long total, int c, int ctas) {
+  return total * c / ctas;
+}
+__device__ __forceinline__ int stream_cta_of(long long total, long long u, int ctas) {
+  return static_cast<int>((static_cast<long long>(ctas) * (u + 1) + total - 1) / total - 1);
+}
+
+// (b, h, k) of unit u, from the block-count prefix sums (b with no blocks
+// are skipped because the largest b with hkv*prefix[b] <= u is taken).
+__device__ __forceinline__ void stream_locate(const int* prefix, int batch, int hkv, long long u,
+                                              int& b, int& h, int& k) {
+  int lo = 0, hi = batch - 1;
+  while (lo < hi) {
+    const int mid = (lo + hi + 1) >> 1;
+    if (static_cast<long long>(hkv) * prefix[mid] <= u) lo = mid;
+    else hi = mid - 1;
+  }
+  b = lo;
+  const int nb = prefix[b + 1] - prefix[b];
+  const long long r = u - static_cast<long long>(hkv) * prefix[b];
+  h = static_cast<int>(r / nb);
+  k = static_cast<int>(r - static_cast<long long>(h) * nb);
+}
+
+__device__ __forceinline__ void stream_next(const int* prefix, int batch, int hkv, int& b, int& h,
+                                            int& k) {
+  k = 0;
+  if (++h == hkv) {
+    h = 0;
+    do {
+      ++b;
+    } while (b < batch && prefix[b + 1] == prefix[b]);
+  }
+}
+
+// prefix[b] = sum_{b' < b} ceil(L_b' / bs) for b in [0, batch]; all threads.
+template <int BS>
+__device__ __forceinline__ void block_count_prefix(int* prefix, int* scan, int batch,
+                                                   const DecodeArgs& a, bool report) {
+  const int t = threadIdx.x;
+  const int per = (batch + kThreads - 1) / kThreads;
+  const int lo = min(batch, t * per);
+  const int hi = min(batch, lo + per);
+  int sum = 0;
+  for (int i = lo; i < hi; ++i) {
+    const int len = effective_len(__ldg(a.seq_lens + i), BS, a, report);
+    const int nb = (len + BS - 1) / BS;
+    prefix[i] = nb;
+    sum += nb;
+  }
+  scan[t] = sum;
+  __syncthreads();
+  if (t < 32) {  // exclusive scan of the kThreads partial sums by one warp
+    constexpr int kPer = (kThreads + 31) / 32;
+    int v[kPer];
+    int run = 0;
+#pragma unroll
+    for (int e = 0; e < kPer; ++e) {
+      const int idx = t * kPer + e;
+      v[e] = idx < kThreads ? scan[idx] : 0;
+      run += v[e];
+    }
+    int incl = run;
+#pragma unroll
+    for (int off = 1; off < 32; off <<= 1) {
+      const int y = __shfl_up_sync(kFull, incl, off);
+      if (t >= off) incl += y;
+    }
+    int excl = incl - run;
+#pragma unroll
+    for (int e = 0; e < kPer; ++e) {
+      const int idx = t * kPer + e;
+      if (idx < kThreads) scan[idx] = excl;
+      excl += v[e];
+    }
+    if (t == 31) scan[kThreads] = incl;  // grand total
+  }
+  __syncthreads();
+  int run = scan[t];
+  for (int i = lo; i < hi; ++i) {
+    const int nb = prefix[i];
+    prefix[i] = run;
+    run += nb;
+  }
+  if (t == 0) prefix[batch] = scan[kThreads];
+  __syncthreads();
+}
+
+__device__ __forceinline__ void consumer_bar() {
+  asm volatile("bar.sync 1, %0;" ::"n"(kConsumerWarps * 32) : "memory");
+}
+
+template <int D, int BS, int VAR, int G>
+__global__ void __launch_bounds__(kThreads, kStreamCtasPerSm)
+    paged_decode_stream_kernel(const __grid_constant__ CUtensorMap kv_map, const DecodeArgs a,
+                               int batch) {
+  using geo = Geo<D, BS>;
+  using sm = StreamSmem<D, BS, G>;
+  extern __shared__ uint8_t smem_raw[];
+  const uint32_t raw_base = smem_u32(smem_raw);
+  const uint32_t pad = ((raw_base + 1023u) & ~1023u) - raw_base;
+  uint8_t* smem = smem_raw + pad;
+  const uint32_t sbase = raw_base + pad;
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const int g = a.group;
+  const int hkv = a.num_kv_heads;
+  const int ctas = gridDim.x;
+  const uint32_t bar_full = sbase + sm::kBar;
+  const uint32_t bar_empty = bar_full + 8 * geo::kStages;
+  int* last_round = reinterpret_cast<int*>(smem + sm::kMisc);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + sm::kMisc + 4 * geo::kStages);
+  int* prefix = reinterpret_cast<int*>(smem + sm::kPrefix);
+
+  if (threadIdx.x == 0) {  // shared memory only: may overlap the previous grid
+    for (int s = 0; s < geo::kStages; ++s) {
+      mbar_init(bar_full + 8 * s, 1);
+      mbar_init(bar_empty + 8 * s, 1);
+      last_round[s] = -1;
+    }
+    *abort_flag = 0;
+    fence_barrier_init();
+  }
+  pdl_trigger();
+  pdl_wait();  // every global access below comes after the previous grid
+  block_count_prefix<BS>(prefix, reinterpret_cast<int*>(smem + sm::kScan), batch, a,
+                         blockIdx.x == 0);
+  if (blockIdx.x == 0)
+    for (int i = threadIdx.x; i <= batch; i += kThreads) a.stream_prefix[i] = prefix[i];
+  const long long total = static_cast<long long>(hkv) * prefix[batch];
+  const long long u_begin = stream_begin(total, blockIdx.x, ctas);
+  const long long u_end = stream_begin(total, blockIdx.x + 1, ctas);
+  if (u_begin >= u_end) return;  // uniform: this CTA has no units
+
+  [[maybe_unused]] MmaConsumer<D, BS> mc;
+  [[maybe_unused]] CudaCoreConsumer<D, BS, (G > 0 ? G : 1)> cc;
+  if (warp == kConsumerWarps) {
+    // ------------------------------------------------------------ producer
+    if (lane == 0) prefetch_tensor_map(&kv_map);
+    int b, h, k;
+    stream_locate(prefix, batch, hkv, u_begin, b, h, k);
+    long long u = u_begin;
+    int i = 0;  // running block index in this CTA
+    bool stop = false;
+    while (u < u_end && !stop) {
+      const int nb = prefix[b + 1] - prefix[b];
+      const int cnt = static_cast<int>(min(static_cast<long long>(nb - k), u_end - u));
+      const int32_t* trow = a.block_tables + static_cast<size_t>(b) * a.max_blocks_per_seq + k;
+      for (int base = 0; base < cnt && !stop; base += 32) {
+        int phys = 0;
+        if (base + lane < cnt) {
+          phys = __ldg(trow + base + lane);
+          if (static_cast<unsigned>(phys) >= static_cast<unsigned>(a.num_blocks)) {
+            flag_error(a.err, PA_DEVERR_BLOCK_ID);
+            phys = 0;  // read a valid block instead; the result is flagged as wrong
+          }
+        }
+        const int n32 = min(32, cnt - base);
+        for (int j = 0; j < n32; ++j) {
+          const int pb = __shfl_sync(kFull, phys, j);
+          int failed = 0;
+          if (lane == 0) {
+            const int ii = i + base + j;
+            const int s = ii % geo::kStages;
+            const int round = ii / geo::kStages;
+            if (!mbar_wait(bar_empty + 8 * s, (round & 1) ^ 1)) {
+              flag_error(a.err, PA_DEVERR_WAIT_TIMEOUT);
+              *abort_flag = 1;
+              failed = 1;
+            } else {
+              const uint32_t fb = bar_full + 8 * s;
+              mbar_arrive_expect_tx(fb, geo::kStageBytes);
+              const uint32_t dst = sbase + s * geo::kStageBytes;
+#pragma unroll
+              for (int x = 0; x < geo::kRegions; ++x)
+                tma_load_3d(dst + x * geo::kRegionBytes, &kv_map, fb, x * 64, h * BS, 2 * pb);
+              last_round[s] = round;
+            }
+          }
+          if (__shfl_sync(kFull, failed, 0)) stop = true;
+          if (stop) break;
+        }
+      }
+      i += cnt;
+      u += cnt;
+      stream_next(prefix, batch, hkv, b, h, k);
+    }
+  } else {
+    // ----------------------------------------------------------- consumers
+    float* pbuf = reinterpret_cast<float*>(smem + sm::kPbuf) + warp * BS * (G > 0 ? G : 1);
+    float* o_all = reinterpret_cast<float*>(smem + sm::kEpi);
+    float* m_all = reinterpret_cast<float*>(smem + sm::kEpi + geo::kEpiO);
+    float* l_all = m_all + kConsumerWarps * kMaxGroup;
+    int b, h, k;
+    stream_locate(prefix, batch, hkv, u_begin, b, h, k);
+    long long u = u_begin;
+    int i = 0;
+    int seg = 0;
+    while (u < u_end) {
+      const int nb = prefix[b + 1] - prefix[b];
+      const int cnt = static_cast<int>(min(static_cast<long long>(nb - k), u_end - u));
+      const bool complete = (k == 0 && cnt == nb);
+      const size_t head0 = static_cast<size_t>(b) * a.num_q_heads + static_cast<size_t>(h) * g;
+      const int len = effective_len(__ldg(a.seq_lens + b), BS, a, false);
+      const int last_valid = len - (nb - 1) * BS;
+      const __nv_bfloat16* qrow = a.q + head0 * D;
+      if constexpr (VAR == kMma) mc.init(qrow, g, lane);
+      else cc.init(qrow, lane);
+      // this warp's blocks of the segment: running indices i..i+cnt-1 that are
+      // congruent to the warp number
+      for (int ii = i + ((warp - i % kConsumerWarps + kConsumerWarps) % kConsumerWarps);
+           ii < i + cnt; ii += kConsumerWarps) {
+        if (*abort_flag) break;
+        const int s = ii % geo::kStages;
+        if (!mbar_wait(bar_full + 8 * s, (ii / geo::kStages) & 1)) {
+          if (lane == 0) {
+            flag_error(a.err, PA_DEVERR_WAIT_TIMEOUT);
+            *abort_flag = 1;
+          }
+          break;
+        }
+        const uint32_t sb = sbase + s * geo::kStageBytes;
+        const int valid = (k + (ii - i) == nb - 1) ? last_valid : BS;
+        consume_block<D, BS, VAR, G>(mc, cc, sb, pbuf, valid, a.scale_log2, lane);
+        __syncwarp();
+        if (lane == 0) mbar_arrive(bar_empty + 8 * s);
+      }
+      // ---- segment epilogue: merge the four warps' states
+      {
+        float* o_s = o_all + warp * kMaxGroup * geo::kOStride;
+        if constexpr (VAR == kMma) mc.store(o_s, m_all + warp * kMaxGroup, l_all + warp * kMaxGroup, lane);
+        else cc.store(o_s, m_all + warp * kMaxGroup, l_all + warp * kMaxGroup, lane);
+      }
+      consumer_bar();
+      if (*abort_flag == 0) {
+        const int slot = (seg == 0) ? 0 : 1;
+        const size_t prow = (static_cast<size_t>(blockIdx.x) * 2 + slot) * g;
+        for (int idx = threadIdx.x; idx < g * D / 2; idx += kConsumerWarps * 32) {
+          const int j = (2 * idx) / D;
+          const int d = (2 * idx) % D;
+          float mm = -INFINITY;
+#pragma unroll
+          for (int w = 0; w < kConsumerWarps; ++w) mm = fmaxf(mm, m_all[w * kMaxGroup + j]);
+          float ll = 0.f, v0 = 0.f, v1 = 0.f;
+#pragma unroll
+          for (int w = 0; w < kConsumerWarps; ++w) {
+            const float mw = m_all[w * kMaxGroup + j];
+            const float f = (mw == -INFINITY) ? 0.f : exp2f(mw - mm);
+            const float* ow = o_all + (w * kMaxGroup + j) * geo::kOStride + d;
+            ll = fmaf(f, l_all[w * kMaxGroup + j], ll);
+            v0 = fmaf(f, ow[0], v0);
+            v1 = fmaf(f, ow[1], v1);
+          }
+          if (complete) {
+            const float inv = 1.f / ll;
+            *reinterpret_cast<__nv_bfloat162*>(a.out + (head0 + j) * D + d) =
+                __floats2bfloat162_rn(v0 * inv, v1 * inv);
+          } else {
+            *reinterpret_cast<float2*>(a.part_o + (prow + j) * D + d) = make_float2(v0, v1);
+            if (d == 0) {
+              a.part_m[prow + j] = mm;
+              a.part_l[prow + j] = ll;
+            }
+          }
+        }
+      }
+      consumer_bar();  // the scratch is free for the next segment
+      i += cnt;
+      u += cnt;
+      ++seg;
+      stream_next(prefix, batch, hkv, b, h, k);
+    }
+  }
+  __syncthreads();
+  if (*abort_flag && threadIdx.x == 0) {
+    // unwind: let every issued tile land before the CTA's memory goes away
+    for (int s = 0; s < geo::kStages; ++s)
+      if (last_round[s] >= 0) mbar_wait_bounded(bar_full + 8 * s, last_round[s] & 1, kWaitLimitNs);
+  }
+}
+
+// Merge for the balanced schedule: one warp per (request, query head).  A
+// (b, h) covered by a single CTA was written directly; a (b, h) split across
+// CTAs c_first..c_last is merged from their partial slots (slot 0 when the
+// (b, h) is the CTA's first segment, else slot 1).  CTAs with an empty range
+// (more CTAs than units) wrote nothing and are skipped.  Requests of length
+// 0 get zeros here.  Three dependent memory rounds per warp: the prefix
+// sums, every CTA's (m, l) (one per lane), then all partial O rows at once.
+template <int D>
+__global__ void __launch_bounds__(128) paged_decode_stream_merge_kernel(const DecodeArgs a,
+                                                                        int batch, int ctas) {
+  constexpr int kPer = D / 32;
+  constexpr int kUnroll = 8;
+  pdl_trigger();
+  pdl_wait();
+  const int gw = blockIdx.x * 4 + (threadIdx.x >> 5);
+  const int lane = threadIdx.x & 31;
+  const int hkv = a.num_kv_heads;
+  const int g = a.group;
+  if (gw >= batch * a.num_q_heads) return;
+  const int b = gw / a.num_q_heads;
+  const int qh = gw - b * a.num_q_heads;  // query head
+  const int h = qh / g;                   // its KV head
+  const int j = qh - h * g;               // its place in the group
+  const int* prefix = a.stream_prefix;
+  const int pb0 = prefix[b], pb1 = prefix[b + 1], pall = prefix[batch];
+  const int nb = pb1 - pb0;
+  __nv_bfloat16* o = a.out + static_cast<size_t>(gw) * D + lane * kPer;
+  if (nb == 0) {
+#pragma unroll
+    for (int e = 0; e < kPer; e += 2)
+      *reinterpret_cast<__nv_bfloat162*>(o + e) = __floats2bfloat162_rn(0.f, 0.f);
+    return;
+  }
+  const long long total = static_cast<long long>(hkv) * pall;
+  const long long us = static_cast<long long>(hkv) * pb0 + static_cast<long long>(h) * nb;
+  const int c0 = stream_cta_of(total, us, ctas);
+  const int c1 = stream_cta_of(total, us + nb - 1, ctas);
+  if (c0 == c1) return;  // one CTA held the whole (b, h) and wrote the output
+  // partial row of CTA c for this (b, h) and group member j, or -1 if c holds no units
+  auto row_of = [&](int c) -> long long {
+    const long long cb = stream_begin(total, c, ctas);
+    if (stream_begin(total, c + 1, ctas) <= cb) return -1;
+    return (static_cast<long long>(c) * 2 + (cb >= us ? 0 : 1)) * g + j;
+  };
+  float mm = -INFINITY, den = 0.f;
+  {
+    float ml[4], ll[4];  // lanes cover up to 128 CTAs per pass
+    for (int c00 = c0; c00 <= c1; c00 += 128) {
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {
+        const int c = c00 + q * 32 + lane;
+        const long long r = c <= c1 ? row_of(c) : -1;
+        ml[q] = r >= 0 ? a.part_m[r] : -INFINITY;
+        ll[q] = r >= 0 ? a.part_l[r] : 0.f;
+      }
+      float m2 = fmaxf(fmaxf(ml[0], ml[1]), fmaxf(ml[2], ml[3]));
+#pragma unroll
+      for (int off = 16; off > 0; off >>= 1) m2 = fmaxf(m2, __shfl_xor_sync(kFull, m2, off));
+      const float mnew = fmaxf(mm, m2);
+      float d2 = 0.f;
+#pragma unroll
+      for (int q = 0; q < 4; ++q)
+        if (ml[q] != -INFINITY) d2 = fmaf(exp2f(ml[q] - mnew), ll[q], d2);
+#pragma unroll
+      for (int off = 16; off > 0; off >>= 1) d2 += __shfl_xor_sync(kFull, d2, off);
+      den = (mm == -INFINITY ? 0.f : den * exp2f(mm - mnew)) + d2;
+      mm = mnew;
+    }
+  }
+  float acc[kPer];
+#pragma unroll
+  for (int e = 0; e < kPer; ++e) acc[e] = 0.f;
+#pragma unroll 1
+  for (int cu = c0; cu <= c1; cu += kUnroll) {
+    float v[kUnroll][kPer];
+    float w[kUnroll];
+    bool ok[kUnroll];
+#pragma unroll
+    for (int q = 0; q < kUnroll; ++q) {
+      const int c = cu + q;
+      const long long r = c <= c1 ? row_of(c) : -1;
+      ok[q] = r >= 0;
+      w[q] = 0.f;
+#pragma unroll
+      for (int e = 0; e < kPer; ++e) v[q][e] = 0.f;
+      if (ok[q]) {
+        w[q] = a.part_m[r];
+        const float* op = a.part_o + r * D + lane * kPer;
+        if constexpr (kPer == 4) {
+          const float4 x = *reinterpret_cast<const float4*>(op);
+          v[q][0] = x.x;
+          v[q][1] = x.y;
+          v[q][2] = x.z;
+          v[q][3] = x.w;
+        } else {
+          const float2 x = *reinterpret_cast<const float2*>(op);
+          v[q][0] = x.x;
+          v[q][1] = x.y;
+        }
+      }
+    }
+#pragma unroll
+    for (int q = 0; q < kUnroll; ++q) {
+      if (ok[q]) {
+        const float wq = exp2f(w[q] - mm);
+#pragma unroll
+        for (int e = 0; e < kPer; ++e) acc[e] = fmaf(wq, v[q][e], acc[e]);
+      }
+    }
+  }
+  const float inv = 1.f / den;
+#pragma unroll
+  for (int e = 0; e < kPer; e += 2)
+    *reinterpret_cast<__nv_bfloat162*>(o + e) = __floats2bfloat162_rn(acc[e] * inv, acc[e + 1] * inv);
+}
+
+// --------------------------------------------------------------------------
 // Log-sum-exp merge of the sequence partitions: one warp per (request, head).
 //   M = max_p m_p;  out = sum_p 2^(m_p - M) O_p / sum_p 2^(m_p - M) l_p
-// (m in the log2 domain; O_p unnormalised w.r.t. its own m_p).
+// (m in the log2 domain; O_p unnormalised w.r.t. its own m_p).  The lanes
+// read the partitions' (m, l) in parallel, then the O rows are read eight
+// partitions at a time with all loads in flight: two or three dependent
+// memory round trips per warp instead of one per partition.
 // --------------------------------------------------------------------------
 template <int D, int BS>
 __global__ void __launch_bounds__(128) paged_decode_reduce_kernel(const DecodeArgs a, int batch) {
   constexpr int kPer = D / 32;
+  constexpr int kUnroll = 8;
+  pdl_trigger();
+  pdl_wait();
   const int gw = blockIdx.x * 4 + (threadIdx.x >> 5);
   const int lane = threadIdx.x & 31;
   if (gw >= batch * a.num_q_heads) return;
@@ -617,28 +1069,52 @@ __global__ void __launch_bounds__(128) paged_decode_reduce_kernel(const DecodeAr
   const int nparts = (nblk + a.part_blocks - 1) / a.part_blocks;
   if (nparts <= 1) return;  // the main kernel wrote this output directly
   const size_t base = static_cast<size_t>(gw) * a.max_parts;
+  const float* pm = a.part_m + base;
+  const float* pl = a.part_l + base;
   float mm = -INFINITY;
-  for (int p = lane; p < nparts; p += 32) mm = fmaxf(mm, a.part_m[base + p]);
+  for (int p = lane; p < nparts; p += 32) mm = fmaxf(mm, pm[p]);
 #pragma unroll
   for (int off = 16; off > 0; off >>= 1) mm = fmaxf(mm, __shfl_xor_sync(kFull, mm, off));
+  float den = 0.f;
+  for (int p = lane; p < nparts; p += 32) den = fmaf(exp2f(pm[p] - mm), pl[p], den);
+#pragma unroll
+  for (int off = 16; off > 0; off >>= 1) den += __shfl_xor_sync(kFull, den, off);
   float acc[kPer];
 #pragma unroll
   for (int e = 0; e < kPer; ++e) acc[e] = 0.f;
-  float den = 0.f;
-  for (int p = 0; p < nparts; ++p) {
-    const float w = exp2f(a.part_m[base + p] - mm);
-    den = fmaf(w, a.part_l[base + p], den);
-    const float* op = a.part_o + (base + p) * D + lane * kPer;
-    if constexpr (kPer == 4) {
-      const float4 v = *reinterpret_cast<const float4*>(op);
-      acc[0] = fmaf(w, v.x, acc[0]);
-      acc[1] = fmaf(w, v.y, acc[1]);
-      acc[2] = fmaf(w, v.z, acc[2]);
-      acc[3] = fmaf(w, v.w, acc[3]);
-    } else {
-      const float2 v = *reinterpret_cast<const float2*>(op);
-      acc[0] = fmaf(w, v.x, acc[0]);
-      acc[1] = fmaf(w, v.y, acc[1]);
+  const float* po = a.part_o + base * D + lane * kPer;
+#pragma unroll 1
+  for (int p0 = 0; p0 < nparts; p0 += kUnroll) {
+    float v[kUnroll][kPer];
+    float w[kUnroll];
+#pragma unroll
+    for (int u = 0; u < kUnroll; ++u) {
+      const int p = p0 + u;
+      w[u] = 0.f;
+#pragma unroll
+      for (int e = 0; e < kPer; ++e) v[u][e] = 0.f;
+      if (p < nparts) {
+        w[u] = pm[p];
+        if constexpr (kPer == 4) {
+          const float4 x = *reinterpret_cast<const float4*>(po + static_cast<size_t>(p) * D);
+          v[u][0] = x.x;
+          v[u][1] = x.y;
+          v[u][2] = x.z;
+          v[u][3] = x.w;
+        } else {
+          const float2 x = *reinterpret_cast<const float2*>(po + static_cast<size_t>(p) * D);
+          v[u][0] = x.x;
+          v[u][1] = x.y;
+        }
+      }
+    }
+#pragma unroll
+    for (int u = 0; u < kUnroll; ++u) {
+      if (p0 + u < nparts) {
+        const float wu = exp2f(w[u] - mm);
+#pragma unroll
+        for (int e = 0; e < kPer; ++e) acc[e] = fmaf(wu, v[u][e], acc[e]);
+      }
     }
   }
   const float inv = 1.f / den;
@@ -652,16 +1128,35 @@ __global__ void __launch_bounds__(128) paged_decode_reduce_kernel(const DecodeAr
 // Host side
 // --------------------------------------------------------------------------
 struct Plan {
+  bool stream = false;  // balanced schedule (else the per-partition grid)
   int part_blocks = 1;
   int max_parts = 1;
-  size_t off_m = 0, off_l = 0, bytes = 0;
+  int ctas = 0;  // stream: persistent CTAs
+  size_t off_m = 0, off_l = 0, off_prefix = 0, bytes = 0;
 };
 
 static size_t align256(size_t x) { return (x + 255) & ~static_cast<size_t>(255); }
 
+// partition_tokens == 0 selects the balanced schedule (batches up to
+// kStreamMaxBatch); a positive value selects the per-partition grid with
+// partitions of that many tokens.
 static int make_plan(int batch, int hq, int hkv, int d, int bs, int max_seq_len,
                      int partition_tokens, Plan* plan) {
   const int nblk_max = max_seq_len > 0 ? (max_seq_len + bs - 1) / bs : 1;
+  const int group = hq / hkv;
+  if (partition_tokens == 0 && batch <= kStreamMaxBatch) {
+    const int sms = sm_count() > 0 ? sm_count() : 148;
+    plan->stream = true;
+    plan->ctas = sms * kStreamCtasPerSm;
+    plan->part_blocks = 1;  // set per call from max_blocks_per_seq
+    plan->max_parts = 1;
+    const size_t rows = static_cast<size_t>(plan->ctas) * 2 * group;
+    plan->off_m = align256(rows * d * sizeof(float));
+    plan->off_l = plan->off_m + align256(rows * sizeof(float));
+    plan->off_prefix = plan->off_l + align256(rows * sizeof(float));
+    plan->bytes = plan->off_prefix + align256((static_cast<size_t>(batch) + 1) * sizeof(int));
+    return PA_OK;
+  }
   int pb;
   if (partition_tokens > 0) {
     if (partition_tokens % bs != 0)
@@ -669,14 +1164,15 @@ static int make_plan(int batch, int hq, int hkv, int d, int bs, int max_seq_len,
                   partition_tokens, bs);
     pb = partition_tokens / bs;
   } else {
-    // 512-token partitions; halve them while the grid would leave the SMs
-    // short of work (few, short requests).
+    // batches above the stream limit: 512-token partitions, halved while the
+    // grid would leave the SMs short of work
     pb = 512 / bs;
     const int sms = sm_count() > 0 ? sm_count() : 148;
     const long long pairs = static_cast<long long>(batch) * hkv;
     while (pb > 4 && pairs * ((nblk_max + pb - 1) / pb) < 4ll * sms) pb /= 2;
   }
   pb = pb < 1 ? 1 : pb;
+  plan->stream = false;
   plan->part_blocks = pb;
   plan->max_parts = (nblk_max + pb - 1) / pb;
   if (plan->max_parts > 1) {
@@ -714,14 +1210,38 @@ static int launch_main(const CUtensorMap& map, const DecodeArgs& a, int batch, c
   if (rc != PA_OK) return rc;
   dim3 grid(static_cast<unsigned>(a.max_parts), static_cast<unsigned>(a.num_kv_heads),
             static_cast<unsigned>(batch));
-  kern<<<grid, kThreads, sm::kDynamic, st>>>(map, a);
-  PA_CUDA_TRY(cudaGetLastError());
+  PA_CUDA_TRY(launch_pdl(kern, grid, dim3(kThreads), sm::kDynamic, st, map, a));
+  return PA_OK;
+}
+
+template <int D, int BS, int VAR, int G>
+static int launch_stream(const CUtensorMap& map, const DecodeArgs& a, int batch, int ctas,
+                         cudaStream_t st) {
+  using sm = StreamSmem<D, BS, G>;
+  auto kern = paged_decode_stream_kernel<D, BS, VAR, G>;
+  const int smem = sm::dynamic_bytes(batch);
+  int rc = set_smem_attr(reinterpret_cast<const void*>(kern), smem);
+  if (rc != PA_OK) return rc;
+  PA_CUDA_TRY(launch_pdl(kern, dim3(static_cast<unsigned>(ctas)), dim3(kThreads), smem, st, map, a, batch));
+  const int warps = batch * a.num_q_heads;
+  PA_CUDA_TRY(launch_pdl(paged_decode_stream_merge_kernel<D>, dim3((warps + 3) / 4), dim3(128), 0, st,
+                         a, batch, ctas));
   return PA_OK;
 }
 
 template <int D, int BS>
 static int dispatch(const CUtensorMap& map, const DecodeArgs& a, int batch, int variant,
-                    cudaStream_t st) {
+                    const Plan& plan, cudaStream_t st) {
+  if (plan.stream) {
+    if (variant == kMma) return launch_stream<D, BS, kMma, 0>(map, a, batch, plan.ctas, st);
+    switch (a.group) {
+      case 1: return launch_stream<D, BS, kCudaCore, 1>(map, a, batch, plan.ctas, st);
+      case 2: return launch_stream<D, BS, kCudaCore, 2>(map, a, batch, plan.ctas, st);
+      case 4: return launch_stream<D, BS, kCudaCore, 4>(map, a, batch, plan.ctas, st);
+      default:
+        return fail(PA_ERR_UNSUPPORTED, "pa_decode: CUDA-core variant has no group size %d", a.group);
+    }
+  }
   int rc;
   if (variant == kMma) {
     rc = launch_main<D, BS, kMma, 0>(map, a, batch, st);
@@ -737,8 +1257,8 @@ static int dispatch(const CUtensorMap& map, const DecodeArgs& a, int batch, int 
   if (rc != PA_OK) return rc;
   if (a.max_parts > 1) {
     const int warps = batch * a.num_q_heads;
-    paged_decode_reduce_kernel<D, BS><<<(warps + 3) / 4, 128, 0, st>>>(a, batch);
-    PA_CUDA_TRY(cudaGetLastError());
+    PA_CUDA_TRY(launch_pdl(paged_decode_reduce_kernel<D, BS>, dim3((warps + 3) / 4), dim3(128), 0, st,
+                           a, batch));
   }
   return PA_OK;
 }
@@ -807,15 +1327,16 @@ static int decode_impl(pa_bf16* out, const pa_bf16* q, const pa_bf16* kv_pool,
   a.group = group;
   a.num_blocks = num_blocks;
   a.max_blocks_per_seq = max_blocks;
-  a.part_blocks = plan.part_blocks;
+  a.part_blocks = plan.stream ? max_blocks : plan.part_blocks;
   a.max_parts = plan.max_parts;
   a.scale_log2 = scale * 1.4426950408889634f;
+  a.stream_prefix = plan.stream ? reinterpret_cast<int*>(ws + plan.off_prefix) : nullptr;
 
   cudaStream_t st = static_cast<cudaStream_t>(stream);
-  if (d == 64 && bs == 16) return dispatch<64, 16>(map, a, batch, variant, st);
-  if (d == 64 && bs == 32) return dispatch<64, 32>(map, a, batch, variant, st);
-  if (d == 128 && bs == 16) return dispatch<128, 16>(map, a, batch, variant, st);
-  return dispatch<128, 32>(map, a, batch, variant, st);
+  if (d == 64 && bs == 16) return dispatch<64, 16>(map, a, batch, variant, plan, st);
+  if (d == 64 && bs == 32) return dispatch<64, 32>(map, a, batch, variant, plan, st);
+  if (d == 128 && bs == 16) return dispatch<128, 16>(map, a, batch, variant, plan, st);
+  return dispatch<128, 32>(map, a, batch, variant, plan, st);
 }
 
 }  // namespace pa
@@ -835,7 +1356,7 @@ int pa_decode_workspace_size_ex(int batch, int num_q_heads, int num_kv_heads, in
                  partition_tokens, &plan);
   if (rc != PA_OK) return rc;
   *bytes_out = plan.bytes;
-  if (num_partitions_out) *num_partitions_out = plan.max_parts;
+  if (num_partitions_out) *num_partitions_out = plan.stream ? plan.ctas : plan.max_parts;
   return PA_OK;
 }
 

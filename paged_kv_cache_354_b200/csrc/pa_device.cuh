@@ -4,7 +4,10 @@
 
 #include <cuda.h>
 #include <cuda_bf16.h>
+#include <cuda_runtime.h>
+
 #include <cstdint>
+#include <utility>
 
 #include "pa.h"
 
@@ -26,6 +29,32 @@ __device__ __forceinline__ uint64_t globaltimer_ns() {
   uint64_t t;
   asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
   return t;
+}
+
+// ------------------------------------------- programmatic dependent launch
+// Every kernel of the library is launched with programmatic stream
+// serialisation, so its launch and shared-memory set-up overlap the tail of
+// the kernel before it.  The rule that keeps this safe: a kernel calls
+// pdl_wait() before its first global-memory access (read or write); that
+// wait returns once the preceding grid has completed and its writes are
+// visible.  pdl_trigger() lets the next kernel launch early.
+__device__ __forceinline__ void pdl_wait() { cudaGridDependencySynchronize(); }
+__device__ __forceinline__ void pdl_trigger() { cudaTriggerProgrammaticLaunchCompletion(); }
+
+template <typename... Exp, typename... Act>
+cudaError_t launch_pdl(void (*kernel)(Exp...), dim3 grid, dim3 block, size_t smem,
+                       cudaStream_t stream, Act&&... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kernel, std::forward<Act>(args)...);
 }
 
 // ---------------------------------------------------------------- mbarrier

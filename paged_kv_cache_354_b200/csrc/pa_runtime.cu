@@ -7,6 +7,7 @@
 
 #include <cstdio>
 #include <mutex>
+#include <vector>
 
 #include "pa_device.cuh"
 #include "pa_internal.h"
@@ -74,12 +75,33 @@ int sm_count() {
   return g_sm_count[dev];
 }
 
+// The attribute is set once per (kernel, device) and raised only when a
+// launch needs more, so steady-state launches (and launches recorded into a
+// CUDA graph after a first eager call) make no attribute calls.
 int set_smem_attr(const void* kernel, int bytes) {
+  struct Entry {
+    const void* kernel;
+    int device;
+    int bytes;
+  };
+  static std::vector<Entry> done;
+  int dev;
+  if (current_device(&dev) != PA_OK) return PA_ERR_CUDA;
+  std::lock_guard<std::mutex> lock(g_mu);
+  for (Entry& e : done)
+    if (e.kernel == kernel && e.device == dev && e.bytes >= bytes) return PA_OK;
   cudaError_t e =
       cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
   if (e != cudaSuccess)
     return fail(PA_ERR_CUDA, "cudaFuncSetAttribute(%d bytes smem): %s", bytes,
                 cudaGetErrorString(e));
+  bool found = false;
+  for (Entry& x : done)
+    if (x.kernel == kernel && x.device == dev) {
+      x.bytes = bytes;
+      found = true;
+    }
+  if (!found) done.push_back({kernel, dev, bytes});
   return PA_OK;
 }
 

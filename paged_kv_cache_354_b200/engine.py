@@ -10,14 +10,23 @@ A decode step of a serving loop, in the order the method needs it:
 3. device: ``pa_decode`` attends every request's query over its whole
    cache through the block table.
 
-Host-side staging uses pinned buffers and one copy per array.
+Host-side staging: the allocator writes a step's slots, copy-on-write pairs,
+block tables and lengths straight into one pinned buffer, which reaches the
+device in a single copy.  The device part of a step (cache write, decode,
+merge) can be recorded once into a CUDA graph and replayed every step.
 """
+
+import ctypes
 
 import numpy as np
 import torch
 
-from . import (PA_DECODE_AUTO, PaAlloc, pa_copy_blocks, pa_decode, pa_decode_workspace_size,
-               pa_reshape_and_cache)
+from . import (PA_DECODE_AUTO, PaAlloc, _check, lib, pa_copy_blocks, pa_decode,
+               pa_decode_workspace_size, pa_reshape_and_cache)
+
+
+def _align(n, a=256):
+    return (n + a - 1) // a * a
 
 
 class PagedDecodeCache:
@@ -39,16 +48,36 @@ class PagedDecodeCache:
             self.max_batch, num_q_heads, num_kv_heads, head_dim, block_size, self.max_seq_len,
             partition_tokens)
         self.workspace = torch.empty(max(nbytes, 256), dtype=torch.uint8, device=self.device)
-        # device-side step inputs
-        self.d_tables = torch.zeros((self.max_batch, self.max_blocks), dtype=torch.int32, device=self.device)
-        self.d_lens = torch.zeros(self.max_batch, dtype=torch.int32, device=self.device)
-        self.d_slots = torch.zeros(self.max_batch, dtype=torch.int64, device=self.device)
-        self.d_pairs = torch.zeros((self.max_batch, 2), dtype=torch.int32, device=self.device)
-        # pinned host staging
-        self.h_tables = torch.zeros((self.max_batch, self.max_blocks), dtype=torch.int32).pin_memory()
-        self.h_lens = torch.zeros(self.max_batch, dtype=torch.int32).pin_memory()
-        self.h_slots = torch.zeros(self.max_batch, dtype=torch.int64).pin_memory()
-        self.h_pairs = torch.zeros((self.max_batch, 2), dtype=torch.int32).pin_memory()
+        # one pinned buffer (and its device twin) for a step's metadata:
+        # slots int64[B] | lens int32[B] | pairs int32[B,2] | tables int32[B,MB]
+        b, mb = self.max_batch, self.max_blocks
+        self._layout = {}
+        off = 0
+        for name, dtype, count in (("slots", torch.int64, b), ("lens", torch.int32, b),
+                                   ("pairs", torch.int32, 2 * b), ("tables", torch.int32, b * mb)):
+            self._layout[name] = (off, dtype, count)
+            off += _align(count * torch.empty((), dtype=dtype).element_size())
+        self.meta_bytes = off
+        self.h_meta = torch.zeros(off, dtype=torch.uint8).pin_memory()
+        self.d_meta = torch.zeros(off, dtype=torch.uint8, device=self.device)
+        self.h_slots, self.h_lens, self.h_pairs, self.h_tables = (
+            self._view(self.h_meta, n) for n in ("slots", "lens", "pairs", "tables"))
+        self.s_slots, self.s_lens, self.s_pairs, self.s_tables = (
+            self._view(self.d_meta, n) for n in ("slots", "lens", "pairs", "tables"))
+        self._ptr = {n: ctypes.c_void_p(self.h_meta.data_ptr() + self._layout[n][0]) for n in self._layout}
+        self._ncow = ctypes.c_int(0)
+        self._ids = None
+        self._ids_src = None
+        self.graph = None
+
+    def _view(self, buf, name):
+        off, dtype, count = self._layout[name]
+        t = buf[off:off + count * torch.empty((), dtype=dtype).element_size()].view(dtype)
+        if name == "pairs":
+            t = t.view(-1, 2)
+        elif name == "tables":
+            t = t.view(self.max_batch, self.max_blocks)
+        return t
 
     # ---------------------------------------------------------------- host
     def plan_append(self, seq_ids):
@@ -61,21 +90,54 @@ class PagedDecodeCache:
         tables, lens = self.alloc.block_tables(seq_ids, self.max_blocks)
         return slots, pairs, tables, lens
 
-    def stage(self, slots, pairs, tables, lens, stream=None):
-        """Copy one step's host metadata to the device (pinned, async)."""
-        b = len(slots)
-        npairs = len(pairs)
-        self.h_slots[:b].numpy()[:] = slots
-        self.h_tables[:b].numpy()[:] = tables
-        self.h_lens[:b].numpy()[:] = lens
+    def host_step(self, seq_ids):
+        """Allocator step for one new token per request (host only), written
+        straight into the pinned metadata buffer.  Returns the number of
+        copy-on-write pairs.  ``seq_ids`` must hold max_batch requests."""
+        if self._ids is None or self._ids_src is not seq_ids:
+            self._ids = np.ascontiguousarray(np.asarray(seq_ids, dtype=np.int64))
+            self._ids_src = seq_ids
+            assert len(self._ids) == self.max_batch
+        h = self.alloc._h
+        ids = ctypes.c_void_p(self._ids.ctypes.data)
+        b = self.max_batch
+        _check(lib.pa_alloc_append_batch(h, ids, b, 1, self._ptr["slots"], self._ptr["pairs"], b,
+                                         ctypes.byref(self._ncow)), "pa_alloc_append_batch")
+        _check(lib.pa_alloc_block_tables(h, ids, b, self.max_blocks, self._ptr["tables"], self._ptr["lens"]),
+               "pa_alloc_block_tables")
+        return self._ncow.value
+
+    def upload(self):
+        """One host-to-device copy of the staged metadata (async, pinned)."""
+        self.d_meta.copy_(self.h_meta, non_blocking=True)
+
+    def capture(self, q, k_new, v_new, out):
+        """Record the device part of a step (cache write, decode, merge) on the
+        staged device metadata into a CUDA graph; replay it with ``replay``.
+
+        Call after one ``host_step`` + ``upload`` so the staged slots are
+        real: the eager warm-up run writes the step's own K/V, which the
+        replay writes again."""
+        side = torch.cuda.Stream(device=self.device)
+        side.wait_stream(torch.cuda.current_stream(self.device))
+        with torch.cuda.stream(side):
+            self._device_step(q, k_new, v_new, out)
+        torch.cuda.current_stream(self.device).wait_stream(side)
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g):
+            self._device_step(q, k_new, v_new, out)
+        self.graph = g
+        return g
+
+    def _device_step(self, q, k_new, v_new, out):
+        pa_reshape_and_cache(k_new, v_new, self.pool, self.s_slots)
+        self.decode(q, out, self.s_tables, self.s_lens)
+
+    def replay(self, npairs):
+        """Device part of a staged step: copy-on-write copies (if any), then the graph."""
         if npairs:
-            self.h_pairs[:npairs].numpy()[:] = pairs
-        self.d_slots[:b].copy_(self.h_slots[:b], non_blocking=True)
-        self.d_tables[:b].copy_(self.h_tables[:b], non_blocking=True)
-        self.d_lens[:b].copy_(self.h_lens[:b], non_blocking=True)
-        if npairs:
-            self.d_pairs[:npairs].copy_(self.h_pairs[:npairs], non_blocking=True)
-        return npairs
+            pa_copy_blocks(self.pool, self.s_pairs[:npairs])
+        self.graph.replay()
 
     # -------------------------------------------------------------- device
     def run(self, q, k_new, v_new, out, slots, tables, lens, pairs=None, max_seq_len=None):

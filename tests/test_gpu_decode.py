@@ -69,6 +69,32 @@ def test_split_k_partitions(partition_blocks, variant):
           partition_tokens=partition_blocks * bs)
 
 
+@pytest.mark.parametrize("lens", [
+    [1, 0, 3],                 # fewer units than CTAs: most CTAs get nothing
+    [0, 0, 0, 0],              # nothing to attend over anywhere
+    [40000],                   # one request cut across every CTA
+    [17, 40000, 0, 5, 2048],   # mixed, with a request split many ways
+])
+@pytest.mark.parametrize("variant", ["mma", "cuda_core"])
+def test_balanced_schedule_edges(lens, variant):
+    check(lens, 8 if variant == "mma" else 4, 2 if variant == "mma" else 4, 64, 16, seed=60 + len(lens),
+          variant=variant)
+
+
+def test_balanced_matches_partition_grid():
+    lens = [3000, 17, 1200, 2049, 5, 640, 2999, 1, 4096, 33]
+    q, pool, _, (t, l) = make_case(lens, 32, 8, 128, 16, seed=61)
+    q, pool = q.cuda(), pool.cuda()
+    bal = run_decode(q, pool, t, l, 0.088, pk.PA_DECODE_MMA, partition_tokens=0)
+    grid = run_decode(q, pool, t, l, 0.088, pk.PA_DECODE_MMA, partition_tokens=512)
+    assert (bal.float() - grid.float()).abs().max().item() <= 2 ** -7
+
+
+def test_batch_above_balanced_limit_uses_grid():
+    lens = list(np.random.default_rng(62).integers(0, 40, size=4100))
+    check(lens, 4, 2, 64, 16, seed=62)
+
+
 def test_split_k_consistency():
     """P=1 and P>1 results agree to fp32-merge rounding, not just to the tolerance."""
     lens = [700, 1024, 64]

@@ -72,10 +72,11 @@ def test_noalloc_matches_pa_decode_on_two_calls(seeds):
 
 
 def test_noalloc_rejects_calls_beyond_its_scratch():
-    # 512 requests x 64 heads x 32768 tokens need far more than the built-in array
-    need, _ = pk.pa_decode_workspace_size(512, 64, 8, 128, 16, 32768)
+    # 8192 requests (above the balanced schedule's batch limit) x 64 heads x
+    # 32768 tokens need far more scratch than the built-in array holds
+    need, _ = pk.pa_decode_workspace_size(8192, 64, 8, 128, 16, 32768)
     assert need > pk.PA_NOALLOC_SCRATCH_BYTES
-    rc = pk.lib.pa_decode_noalloc(None, None, None, None, None, 512, 64, 8, 128, 16, 100000, 2048, 32768,
+    rc = pk.lib.pa_decode_noalloc(None, None, None, None, None, 8192, 64, 8, 128, 16, 100000, 2048, 32768,
                                   0.1, None)
     assert rc == pk.PA_ERR_UNSUPPORTED
     assert "scratch" in pk.lib.pa_last_error_string().decode()
