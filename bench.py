@@ -18,6 +18,7 @@ own pool and allocator), no data-path collective.
 """
 
 import argparse
+import hashlib
 import json
 import math
 import os
@@ -38,6 +39,31 @@ import workloads  # noqa: E402
 METRIC = "paged-decode KV-read GB/s & % of HBM peak; decode seqs/s at Llama-3-8B shape"
 PEAKS_FALLBACK = {"hbm_gbs": 6650.0, "source": "fallback"}
 INPUT_SETS = 4  # distinct q/k/v sets cycled through the steps
+
+
+TRAFFIC_FILE = os.path.join(ROOT, "profiles", "paged_decode_traffic.json")
+DECODE_SOURCES = ("paged_kv_cache_354_b200/csrc/pa_decode.cu", "paged_kv_cache_354_b200/csrc/pa_device.cuh")
+
+
+def decode_source_digest():
+    h = hashlib.sha256()
+    for rel in DECODE_SOURCES:
+        with open(os.path.join(ROOT, rel), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()
+
+
+def captured_traffic(workload, variant, partition_tokens):
+    """DRAM bytes per decode launch from the committed ncu capture, or None
+    when there is none for this configuration or the kernel changed since."""
+    try:
+        with open(TRAFFIC_FILE) as f:
+            entry = json.load(f).get(f"{workload}/{variant}/{partition_tokens}")
+    except Exception:
+        return None
+    if not entry or entry.get("source_sha256") != decode_source_digest():
+        return None
+    return entry["dram_bytes_per_launch"]
 
 
 def load_peaks():
@@ -120,7 +146,7 @@ def decode_bytes(lens, hq, hkv, d, bs):
     return kv + qo + tables, kv
 
 
-def build_cache(name, steps_total, rank, device, prefill=True):
+def build_cache(name, steps_total, rank, device, prefill=True, variant=0, partition_tokens=0):
     """Pool (seeded bf16 N(0,1)), allocator state and request ids of a workload.
 
     With ``prefill`` the beam workload's 256 divergent tokens per beam are
@@ -136,7 +162,8 @@ def build_cache(name, steps_total, rank, device, prefill=True):
     max_len = int(lens0.max()) + (p.prefix_len and 256) + steps_total + 2
     batch = len(lens0) * (p.beams or 1)
     cache = PagedDecodeCache(p.num_blocks, s.num_q_heads, s.num_kv_heads, s.head_dim, s.block_size,
-                             batch, max_len, initial_order=p.initial_order, device=device)
+                             batch, max_len, initial_order=p.initial_order, device=device,
+                             partition_tokens=partition_tokens, variant=variant)
     gen = torch.Generator(device=device)
     gen.manual_seed(workloads.seed_of(name) * 1000 + rank)
     cache.pool.copy_(torch.randn(cache.pool.shape, generator=gen, device=device,
@@ -210,7 +237,9 @@ def run_gpu(args):
     from paged_kv_cache_354_b200 import pa_device_error
 
     K, W = args.steps, args.warmup
-    p, cache, ids, gen = build_cache(args.workload, 2 * (W + K), rank, device)
+    variant = {"auto": 0, "cuda_core": 1, "mma": 2}[args.variant]
+    p, cache, ids, gen = build_cache(args.workload, 2 * (W + K), rank, device, variant=variant,
+                                     partition_tokens=args.partition_tokens)
     batch = len(ids)
     qs, ks, vs = make_inputs(cache, batch, gen, device)
     out = torch.empty_like(qs[0])
@@ -335,6 +364,7 @@ def run_gpu(args):
                                     f"per-partition grid: {cache.num_partitions} partitions"),
                 "l2": f"inputs larger than L2: KV read per step {step_bytes[W][1] / 1e6:.0f} MB > 126 MB",
                 "parallelism": f"dp{world} (independent batches, no collective)",
+                "variant": args.variant,
             },
             "decode_seqs_per_s": round(batch * world * K / (dev_ms * 1e-3), 1),
             "frac_of_hbm_peak": round(gbs / world / peaks["hbm_gbs"], 4),
@@ -346,7 +376,9 @@ def run_gpu(args):
                 "unit": "GB/s",
                 "frac": round(achieved / peaks["hbm_gbs"], 4),
                 "peak_source": peaks["source"],
-                "traffic": None,
+                "traffic": captured_traffic(args.workload, args.variant, args.partition_tokens),
+                "traffic_note": "dram read+write per launch of the main decode kernel from the committed "
+                                "ncu capture; null when none matches the current source",
             },
             "e2e": {
                 "value": round(e2e_bytes_all / (e2e_ms * 1e-3) / 1e9, 2),
@@ -477,6 +509,10 @@ def main():
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--workload", default="llama8b", choices=workloads.NAMES)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--variant", default="auto", choices=["auto", "mma", "cuda_core"],
+                    help="decode consumer: auto (tensor cores for GQA groups >= 4), or forced")
+    ap.add_argument("--partition-tokens", type=int, default=0,
+                    help="0 = balanced schedule; N > 0 = per-partition grid of N-token partitions")
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     args = ap.parse_args()
