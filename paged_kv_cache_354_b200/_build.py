@@ -51,8 +51,8 @@ def _stale(target, deps):
     return any(os.path.getmtime(d) > t for d in deps)
 
 
-def _compile(src, force, verbose, extra):
-    obj = os.path.join(OBJDIR, os.path.basename(src) + ".o")
+def _compile(src, force, verbose, extra, objdir=OBJDIR):
+    obj = os.path.join(objdir, os.path.basename(src) + ".o")
     if not force and not _stale(obj, [src, __file__] + _headers()):
         return obj
     cmd = [nvcc(), "-c", src, "-o", obj] + ARCH + COMMON + extra
@@ -68,18 +68,21 @@ def _compile(src, force, verbose, extra):
     return obj
 
 
-def build(force=False, verbose=False, extra=()):
-    """Compile every source under csrc/ and link libpa.so; returns its path."""
-    os.makedirs(OBJDIR, exist_ok=True)
+def build(force=False, verbose=False, extra=(), lib=LIB, objdir=OBJDIR):
+    """Compile every source under csrc/ and link a shared library (libpa.so
+    next to this file unless ``lib`` says otherwise); returns its path.
+    ``extra`` nvcc flags (e.g. -D tuning overrides) should go with their own
+    ``lib`` and ``objdir``."""
+    os.makedirs(objdir, exist_ok=True)
     srcs = _sources()
     with cf.ThreadPoolExecutor(max_workers=min(8, len(srcs))) as ex:
-        objs = list(ex.map(lambda s: _compile(s, force, verbose, list(extra)), srcs))
-    if force or _stale(LIB, objs):
-        cmd = [nvcc(), "-shared", "-o", LIB] + objs + ARCH + ["-Xcompiler", "-fPIC"]
+        objs = list(ex.map(lambda s: _compile(s, force, verbose, list(extra), objdir), srcs))
+    if force or _stale(lib, objs):
+        cmd = [nvcc(), "-shared", "-o", lib] + objs + ARCH + ["-Xcompiler", "-fPIC"]
         res = subprocess.run(cmd, capture_output=True, text=True)
         if res.returncode != 0:
             raise RuntimeError(f"link failed:\n{res.stdout}\n{res.stderr}")
-    return LIB
+    return lib
 
 
 def main(argv=None):

@@ -52,6 +52,7 @@ struct Geo {
   static constexpr int kStageBytes = kRegions * kRegionBytes;  // one block of one head
   static constexpr int kStages = (kStageBytes <= 8192) ? 8 : 4;
   static constexpr int kStageSmem = kStages * kStageBytes;
+  // stage s must always go to warp s % warps (see StreamSmem::kStages)
   static_assert(kStages % kConsumerWarps == 0, "stage s must always go to warp s % warps");
   // epilogue scratch aliased on the stage ring; head rows padded by 4
   // floats so the tensor-core store pattern hits 32 distinct banks
@@ -631,15 +632,32 @@ __global__ void __launch_bounds__(kThreads, (VAR == kMma || G <= 2) ? 3 : 2)
 // can be) writes an fp32 partial into slot 0 (first) or 1 (last) of the CTA,
 // merged afterwards by paged_decode_stream_merge_kernel.
 // --------------------------------------------------------------------------
-constexpr int kStreamCtasPerSm = 2;
+// Build-time tuning of the balanced schedule: CTAs per SM and bytes of TMA
+// ring per CTA (the stage count is the ring size over one block's bytes).
+#ifndef PA_STREAM_CTAS_PER_SM
+#define PA_STREAM_CTAS_PER_SM 2
+#endif
+#ifndef PA_STREAM_RING_BYTES
+#define PA_STREAM_RING_BYTES 65536
+#endif
+constexpr int kStreamCtasPerSm = PA_STREAM_CTAS_PER_SM;
 constexpr int kStreamMaxBatch = 4096;  // the prefix table lives in shared memory
 
 template <int D, int BS, int G>
 struct StreamSmem {
   using geo = Geo<D, BS>;
-  static constexpr int kBar = geo::kStageSmem;                   // full[S], empty[S]
-  static constexpr int kMisc = kBar + 16 * geo::kStages;         // last_round[S], abort
-  static constexpr int kScan = (kMisc + 4 * geo::kStages + 4 + 15) & ~15;  // scan scratch
+  // Stage s must always be consumed by warp s % kConsumerWarps: a warp then
+  // takes a stage's rounds one after the other, so a parity wait (which
+  // only tells the current phase from the previous one) never runs two
+  // rounds ahead.  Hence a whole multiple of the consumer warp count.
+  static constexpr int kRingStages =
+      (PA_STREAM_RING_BYTES / geo::kStageBytes) / kConsumerWarps * kConsumerWarps;
+  static constexpr int kStages = kRingStages > kConsumerWarps ? kRingStages : kConsumerWarps;
+  static_assert(kStages >= kConsumerWarps && kStages % kConsumerWarps == 0,
+                "stages must be a positive multiple of the consumer warps");
+  static constexpr int kBar = kStages * geo::kStageBytes;         // full[S], empty[S]
+  static constexpr int kMisc = kBar + 16 * kStages;               // last_round[S], abort
+  static constexpr int kScan = (kMisc + 4 * kStages + 4 + 15) & ~15;  // scan scratch
   static constexpr int kPbuf = kScan + (kThreads + 4) * 4;       // CUDA-core p tiles
   static constexpr int kPbufBytes = kConsumerWarps * BS * (G > 0 ? G : 1) * 4;
   static constexpr int kEpi = (kPbuf + kPbufBytes + 15) & ~15;   // per-warp O, m, l
@@ -758,13 +776,13 @@ __global__ void __launch_bounds__(kThreads, kStreamCtasPerSm)
   const int hkv = a.num_kv_heads;
   const int ctas = gridDim.x;
   const uint32_t bar_full = sbase + sm::kBar;
-  const uint32_t bar_empty = bar_full + 8 * geo::kStages;
+  const uint32_t bar_empty = bar_full + 8 * sm::kStages;
   int* last_round = reinterpret_cast<int*>(smem + sm::kMisc);
-  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + sm::kMisc + 4 * geo::kStages);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + sm::kMisc + 4 * sm::kStages);
   int* prefix = reinterpret_cast<int*>(smem + sm::kPrefix);
 
   if (threadIdx.x == 0) {  // shared memory only: may overlap the previous grid
-    for (int s = 0; s < geo::kStages; ++s) {
+    for (int s = 0; s < sm::kStages; ++s) {
       mbar_init(bar_full + 8 * s, 1);
       mbar_init(bar_empty + 8 * s, 1);
       last_round[s] = -1;
@@ -812,8 +830,8 @@ __global__ void __launch_bounds__(kThreads, kStreamCtasPerSm)
           int failed = 0;
           if (lane == 0) {
             const int ii = i + base + j;
-            const int s = ii % geo::kStages;
-            const int round = ii / geo::kStages;
+            const int s = ii % sm::kStages;
+            const int round = ii / sm::kStages;
             if (!mbar_wait(bar_empty + 8 * s, (round & 1) ^ 1)) {
               flag_error(a.err, PA_DEVERR_WAIT_TIMEOUT);
               *abort_flag = 1;
@@ -862,8 +880,8 @@ __global__ void __launch_bounds__(kThreads, kStreamCtasPerSm)
       for (int ii = i + ((warp - i % kConsumerWarps + kConsumerWarps) % kConsumerWarps);
            ii < i + cnt; ii += kConsumerWarps) {
         if (*abort_flag) break;
-        const int s = ii % geo::kStages;
-        if (!mbar_wait(bar_full + 8 * s, (ii / geo::kStages) & 1)) {
+        const int s = ii % sm::kStages;
+        if (!mbar_wait(bar_full + 8 * s, (ii / sm::kStages) & 1)) {
           if (lane == 0) {
             flag_error(a.err, PA_DEVERR_WAIT_TIMEOUT);
             *abort_flag = 1;
@@ -925,7 +943,7 @@ __global__ void __launch_bounds__(kThreads, kStreamCtasPerSm)
   __syncthreads();
   if (*abort_flag && threadIdx.x == 0) {
     // unwind: let every issued tile land before the CTA's memory goes away
-    for (int s = 0; s < geo::kStages; ++s)
+    for (int s = 0; s < sm::kStages; ++s)
       if (last_round[s] >= 0) mbar_wait_bounded(bar_full + 8 * s, last_round[s] & 1, kWaitLimitNs);
   }
 }
