@@ -502,6 +502,105 @@ def run_reference(args):
     print(json.dumps(line), flush=True)
 
 
+# --------------------------------------------------------------------------
+# studies of the pages' context claims (not the headline line)
+# --------------------------------------------------------------------------
+MAX_CONTEXT = {"tiny": 65, "llama8b": 4096, "long": 32768, "beam": 2306, "mixed": 8192}
+
+
+def study_memory_waste():
+    """Slots held vs tokens stored: contiguous max-context reservation against
+    the paged allocator's actual state, per workload (host only).
+
+    "Paged attention in LLMs", sections "Why the memory gets wasted" and "Why
+    this helps so much"; the quiz page's table row "Wasted memory".  The
+    contiguous layout reserves the workload's maximum context per request and
+    stores every beam's copy of a shared prefix; the paged numbers come from
+    the C++ allocator after the workload's events.
+    """
+    import paged_kv_cache_354_b200 as pk
+
+    for name in workloads.NAMES:
+        p = workloads.plan(name)
+        a = pk.PaAlloc(p.num_blocks, p.shape.block_size, p.initial_order)
+        ids = workloads.populate(a, p)
+        if p.append_tokens:
+            a.append_batch(ids, p.append_tokens)
+        st = a.stats()
+        bs = p.shape.block_size
+        reserved = len(ids) * MAX_CONTEXT[name]
+        line = {
+            "study": "memory_waste", "workload": name, "requests": len(ids), "block_size": bs,
+            "tokens": st["tokens"],
+            "contiguous_reserved_slots": reserved,
+            "contiguous_waste_frac": round(1 - st["tokens"] / reserved, 4),
+            "paged_logical_slots": st["logical_slots"],
+            "paged_internal_waste_frac": round(1 - st["tokens"] / st["logical_slots"], 4),
+            "paged_physical_slots": st["physical_blocks"] * bs,
+            "paged_physical_over_tokens": round(st["physical_blocks"] * bs / st["tokens"], 4),
+            "max_internal_waste_per_request": bs - 1,
+        }
+        print(json.dumps(line), flush=True)
+
+
+def study_page_table(iters=30):
+    """pa_decode on the workload's scattered block tables vs on identity
+    tables (each request's blocks physically consecutive, same lengths and
+    pool format): the cost the block-table indirection adds to the kernel
+    (quiz page, comparison table row "Kernel overhead": small, <5%)."""
+    import torch
+
+    import paged_kv_cache_354_b200 as pk
+    from paged_kv_cache_354_b200.engine import PagedDecodeCache
+
+    dev = torch.device("cuda", torch.cuda.current_device())
+    for name in ("llama8b", "mixed", "long"):
+        p = workloads.plan(name)
+        s = p.shape
+        res = {}
+        for layout, order in (("scattered", p.initial_order), ("identity", np.arange(p.num_blocks))):
+            cache = PagedDecodeCache(p.num_blocks, s.num_q_heads, s.num_kv_heads, s.head_dim, s.block_size,
+                                     len(p.seq_lens), int(max(p.seq_lens)) + 2, initial_order=order, device=dev)
+            gen = torch.Generator(device=dev)
+            gen.manual_seed(workloads.seed_of(name))
+            cache.pool.copy_(torch.randn(cache.pool.shape, generator=gen, device=dev).bfloat16())
+            if layout == "scattered":
+                ids = workloads.populate(cache.alloc, p)
+            else:  # requests filled in order from an untouched pool (no churn)
+                ids = list(range(len(p.seq_lens)))
+                for sid in ids:
+                    cache.alloc.add_seq(sid)
+                    cache.alloc.append(sid, int(p.seq_lens[sid]))
+            tables, lens = cache.alloc.block_tables(ids, cache.max_blocks)
+            if layout == "identity":
+                flat = np.concatenate([t[: -(-int(n) // s.block_size)] for t, n in zip(tables, lens)])
+                assert np.array_equal(np.diff(flat), np.ones(len(flat) - 1)), "identity layout not consecutive"
+            q = torch.randn((len(ids), s.num_q_heads, s.head_dim), generator=gen, device=dev).bfloat16()
+            out = torch.empty_like(q)
+            d_t, d_l = torch.as_tensor(tables, device=dev), torch.as_tensor(lens, device=dev)
+            for _ in range(3):
+                cache.decode(q, out, d_t, d_l)
+            torch.cuda.synchronize()
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record()
+            for _ in range(iters):
+                cache.decode(q, out, d_t, d_l)
+            e1.record()
+            torch.cuda.synchronize()
+            us = e0.elapsed_time(e1) / iters * 1e3
+            nbytes = decode_bytes(lens, s.num_q_heads, s.num_kv_heads, s.head_dim, s.block_size)[0]
+            res[layout] = (us, nbytes / us / 1e3)
+            del cache
+            torch.cuda.empty_cache()
+        print(json.dumps({
+            "study": "page_table_overhead", "workload": name,
+            "scattered_us": round(res["scattered"][0], 2), "identity_us": round(res["identity"][0], 2),
+            "scattered_gbs": round(res["scattered"][1], 1), "identity_gbs": round(res["identity"][1], 1),
+            "overhead_frac": round(res["scattered"][0] / res["identity"][0] - 1, 4),
+            "iters": iters}), flush=True)
+    assert pk.pa_device_error() == 0
+
+
 def main():
     ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
     ap.add_argument("--gpus", type=int, default=1)
@@ -511,6 +610,8 @@ def main():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--variant", default="auto", choices=["auto", "mma", "cuda_core"],
                     help="decode consumer: auto (tensor cores for GQA groups >= 4), or forced")
+    ap.add_argument("--study", choices=["memory-waste", "page-table"],
+                    help="print the study's JSON lines instead of the benchmark line")
     ap.add_argument("--partition-tokens", type=int, default=0,
                     help="0 = balanced schedule; N > 0 = per-partition grid of N-token partitions")
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
@@ -518,7 +619,11 @@ def main():
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be at least 3")
-    if args.impl == "reference":
+    if args.study == "memory-waste":
+        study_memory_waste()
+    elif args.study == "page-table":
+        study_page_table()
+    elif args.impl == "reference":
         run_reference(args)
     else:
         run_gpu(args)

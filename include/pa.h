@@ -287,6 +287,17 @@ int pa_alloc_block_table(const pa_alloc* a, int64_t seq_id, int32_t* out, int ca
  * [num_seqs].  A table longer than max_blocks_per_seq: PA_ERR_INVALID. */
 int pa_alloc_block_tables(const pa_alloc* a, const int64_t* seq_ids, int num_seqs,
                           int max_blocks_per_seq, int32_t* tables_out, int32_t* seq_lens_out);
+/* Occupancy of the pool ("Paged attention in LLMs", sections "A worked
+ * example" and "Why this helps so much": slots held vs used).
+ * stats_out host int64 [5]:
+ *   [0] tokens stored    = sum of the live requests' lengths
+ *   [1] logical slots    = sum over live requests of table length * block_size
+ *   [2] physical blocks  = blocks with refcount > 0 (shared blocks once)
+ *   [3] live requests
+ *   [4] free blocks
+ * Internal waste = [1] - [0] (at most block_size-1 per request); slots saved
+ * by sharing = [1] - [2]*block_size. */
+int pa_alloc_stats(const pa_alloc* a, int64_t* stats_out);
 /* Full state for comparison: free_list_out host int32 [num_blocks] gets the
  * free blocks in the order the next pops return them (*num_free_out of
  * them); refcounts_out host int32 [num_blocks]. */

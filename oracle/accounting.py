@@ -49,3 +49,26 @@ def contiguous_fits(free_gaps, request_slots):
 def paged_fits(num_free_blocks, request_slots, block_size):
     """Any free block fits any request: only the block count matters."""
     return num_free_blocks * block_size >= request_slots
+
+
+def allocator_stats(alloc):
+    """Occupancy of a block allocator model, counted from its tables.
+
+    tokens          -- sum of the live requests' lengths
+    logical_slots   -- sum over requests of (blocks in its table) * block_size
+    physical_blocks -- distinct physical blocks referenced by any table
+    live_requests   -- number of requests
+    free_blocks     -- blocks on the free list
+    Internal waste is logical_slots - tokens ("Why this helps so much": the
+    tail of each request's last block); sharing saves logical_slots -
+    physical_blocks * block_size ("Sharing blocks").
+    """
+    ids = alloc.seq_ids()
+    tables = [alloc.block_table(s) for s in ids]
+    return {
+        "tokens": sum(alloc.seq_len(s) for s in ids),
+        "logical_slots": sum(len(t) for t in tables) * alloc.block_size,
+        "physical_blocks": len({b for t in tables for b in t}),
+        "live_requests": len(ids),
+        "free_blocks": alloc.num_free(),
+    }

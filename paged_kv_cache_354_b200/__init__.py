@@ -73,6 +73,7 @@ _SIGNATURES = {
     "pa_alloc_block_table": (_I, [_P, _I64, _P, _I, _P]),
     "pa_alloc_block_tables": (_I, [_P, _P, _I, _I, _P, _P]),
     "pa_alloc_dump": (_I, [_P, _P, _P, _P]),
+    "pa_alloc_stats": (_I, [_P, _P]),
 }
 
 
@@ -341,6 +342,13 @@ class PaAlloc:
         _check(lib.pa_alloc_dump(self._h, free.ctypes.data_as(ctypes.c_void_p), ctypes.byref(n),
                                  refs.ctypes.data_as(ctypes.c_void_p)), "pa_alloc_dump")
         return free[: n.value].tolist(), refs.tolist()
+
+    def stats(self):
+        """dict: tokens, logical_slots, physical_blocks, live_requests, free_blocks."""
+        out = np.zeros(5, dtype=np.int64)
+        _check(lib.pa_alloc_stats(self._h, out.ctypes.data_as(ctypes.c_void_p)), "pa_alloc_stats")
+        keys = ("tokens", "logical_slots", "physical_blocks", "live_requests", "free_blocks")
+        return dict(zip(keys, (int(x) for x in out)))
 
     def free_list(self):
         return self.dump()[0]

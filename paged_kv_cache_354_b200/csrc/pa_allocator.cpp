@@ -285,6 +285,22 @@ int pa_alloc_block_tables(const pa_alloc* a, const int64_t* seq_ids, int num_seq
   return PA_OK;
 }
 
+int pa_alloc_stats(const pa_alloc* a, int64_t* stats_out) {
+  if (a == nullptr || stats_out == nullptr) return pa::fail(PA_ERR_INVALID, "pa_alloc_stats: NULL argument");
+  int64_t tokens = 0, logical = 0;
+  for (const auto& kv : a->seqs) {
+    tokens += kv.second.len;
+    logical += static_cast<int64_t>(kv.second.table.size()) * a->block_size;
+  }
+  const int64_t free_blocks = static_cast<int64_t>(a->free_stack.size());
+  stats_out[0] = tokens;
+  stats_out[1] = logical;
+  stats_out[2] = a->num_blocks - free_blocks;
+  stats_out[3] = static_cast<int64_t>(a->seqs.size());
+  stats_out[4] = free_blocks;
+  return PA_OK;
+}
+
 int pa_alloc_dump(const pa_alloc* a, int32_t* free_list_out, int* num_free_out,
                   int32_t* refcounts_out) {
   if (a == nullptr || free_list_out == nullptr || num_free_out == nullptr || refcounts_out == nullptr)

@@ -20,9 +20,12 @@ GOLDEN = json.load(open(os.path.join(os.path.dirname(__file__), "golden", "worke
 
 
 def same_state(cpp, ref):
+    from oracle.accounting import allocator_stats
+
     free, refs = cpp.dump()
     assert free == ref.free_list()
     assert refs == ref.refcounts()
+    assert cpp.stats() == allocator_stats(ref)
     for sid in ref.seq_ids():
         assert cpp.block_table(sid) == ref.block_table(sid)
         assert cpp.seq_len(sid) == ref.seq_len(sid)

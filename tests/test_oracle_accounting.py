@@ -70,3 +70,23 @@ def test_waste_bound_brute_force():
 def test_contiguous_rejects_overflow():
     with pytest.raises(ValueError):
         accounting.contiguous(10, 11)
+
+
+def test_allocator_stats_worked_example_and_sharing():
+    from oracle.block_allocator import BlockAllocator
+
+    g = GOLDEN["worked_example"]
+    a = BlockAllocator(10, g["paged"]["block_size"])
+    a.add_seq(0)
+    a.append(0, g["reply_tokens"])
+    st = accounting.allocator_stats(a)
+    assert st["tokens"] == g["paged"]["used"]
+    assert st["logical_slots"] == g["paged"]["held"]
+    assert st["logical_slots"] - st["tokens"] == g["paged"]["wasted"]
+    assert st["physical_blocks"] == g["paged"]["blocks"] and st["free_blocks"] == 10 - 3
+    # three forks share every block: logical slots x4, physical unchanged
+    for child in (1, 2, 3):
+        a.fork(0, child)
+    st = accounting.allocator_stats(a)
+    assert st["logical_slots"] == 4 * g["paged"]["held"]
+    assert st["physical_blocks"] == g["paged"]["blocks"] and st["live_requests"] == 4
