@@ -263,28 +263,33 @@ def run_gpu(args):
     torch.cuda.synchronize()
     if world > 1:
         dist.barrier()
-    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(K)]
     start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    from paged_kv_cache_354_b200 import pa_copy_blocks, pa_reshape_and_cache
+
     with ClockSampler(device.index) as clocks:
         start.record(stream)
         for i in range(W, W + K):
             j = i % INPUT_SETS
             if d_pairs[i].shape[0]:
-                from paged_kv_cache_354_b200 import pa_copy_blocks
-
                 pa_copy_blocks(cache.pool, d_pairs[i])
-            from paged_kv_cache_354_b200 import pa_reshape_and_cache
-
             pa_reshape_and_cache(ks[j], vs[j], cache.pool, d_slots[i])
-            ev[i - W][0].record(stream)
             cache.decode(qs[j], out, d_tables[i], d_lens[i])
-            ev[i - W][1].record(stream)
         end.record(stream)
+        torch.cuda.synchronize()
+        # the dominant kernel alone: K back-to-back decode launches (main + merge)
+        # on the last step's inputs, bracketed by events on the launching stream
+        k0, k1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        last = W + K - 1
+        k0.record(stream)
+        for i in range(K):
+            cache.decode(qs[i % INPUT_SETS], out, d_tables[last], d_lens[last])
+        k1.record(stream)
         torch.cuda.synchronize()
     if world > 1:
         dist.barrier()
     dev_ms = start.elapsed_time(end)
-    decode_ms = [a.elapsed_time(b) for a, b in ev]
+    decode_ms = [k0.elapsed_time(k1) / K]
+    decode_bytes_last = step_bytes[last][0]
     bytes_timed = sum(b for b, _ in step_bytes[W:])
     kv_timed = sum(kv for _, kv in step_bytes[W:])
 
@@ -339,8 +344,7 @@ def run_gpu(args):
     if rank == 0:
         peaks = load_peaks()
         gbs = bytes_all / (dev_ms * 1e-3) / 1e9
-        per_launch_bytes = bytes_timed / K
-        achieved = per_launch_bytes / (decode_avg_ms * 1e-3) / 1e9
+        achieved = decode_bytes_last / (decode_avg_ms * 1e-3) / 1e9
         line = {
             "metric": METRIC,
             "value": round(gbs, 2),
@@ -370,7 +374,7 @@ def run_gpu(args):
             "frac_of_hbm_peak": round(gbs / world / peaks["hbm_gbs"], 4),
             "roofline": {
                 "bound": "hbm",
-                "kernel": "pa_decode (main + split-K merge)",
+                "kernel": "pa_decode (main + split-K merge), K back-to-back launches",
                 "achieved": round(achieved, 2),
                 "peak": peaks["hbm_gbs"],
                 "unit": "GB/s",
