@@ -364,7 +364,7 @@ def run_gpu(args):
                 "block_size": cache.bs, "num_blocks": cache.num_blocks,
                 "mean_seq_len": round(float(np.mean(plans[W][3])), 1),
                 "decode_schedule": (f"balanced persistent: {cache.num_partitions} CTAs"
-                                    if cache.partition_tokens == 0 else
+                                    if cache.schedule == "balanced" else
                                     f"per-partition grid: {cache.num_partitions} partitions"),
                 "l2": f"inputs larger than L2: KV read per step {step_bytes[W][1] / 1e6:.0f} MB > 126 MB",
                 "parallelism": f"dp{world} (independent batches, no collective)",
@@ -617,7 +617,8 @@ def main():
     ap.add_argument("--study", choices=["memory-waste", "page-table"],
                     help="print the study's JSON lines instead of the benchmark line")
     ap.add_argument("--partition-tokens", type=int, default=0,
-                    help="0 = balanced schedule; N > 0 = per-partition grid of N-token partitions")
+                    help="0 = library's choice; -1 = balanced schedule; N > 0 = per-partition grid of "
+                         "N-token partitions")
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     args = ap.parse_args()

@@ -152,11 +152,13 @@ int pa_copy_blocks(pa_bf16* kv_pool, const int32_t* block_pairs, int num_pairs,
  *                (fp32 partial outputs and log-sum-exp terms of the
  *                sequence partitions), 256-byte aligned; its contents need
  *                no initialisation.
- * Schedule: batches of up to 4096 requests use a balanced persistent
- * schedule -- two CTAs per SM, each taking an equal contiguous share of all
- * (request, KV head, block) units -- followed by a log-sum-exp merge of the
- * (request, head) pairs cut between CTAs.  Larger batches use one CTA per
- * (request, KV head, 512-token partition) and the same kind of merge.
+ * Schedule: batches of up to 4096 requests with at least ~4 blocks of work
+ * per SM (batch * num_kv_heads * ceil(max_seq_len / block_size) >= 4 * SMs)
+ * use a balanced persistent schedule -- two CTAs per SM, each taking an
+ * equal contiguous share of all (request, KV head, block) units -- followed
+ * by a log-sum-exp merge of the (request, head) pairs cut between CTAs.
+ * Other calls use one CTA per (request, KV head, partition of up to 512
+ * tokens) and the same kind of merge.
  * Supported: head_dim in {64, 128}; block_size in {16, 32}; num_q_heads a
  * multiple of num_kv_heads with group size 1..8.  Others: PA_ERR_UNSUPPORTED.
  * Launches: two kernels (decode + merge); the per-partition schedule skips
@@ -183,14 +185,16 @@ typedef enum pa_decode_variant {
 
 /* pa_decode with explicit choices, for measurement and tests.
  * variant          : pa_decode_variant.
- * partition_tokens : 0 = the built-in schedule (see pa_decode); > 0 = one
- *                    CTA per (request, KV head, partition of this many
- *                    tokens, a multiple of block_size).  The workspace must
- *                    be sized with pa_decode_workspace_size_ex for the same
- *                    value. */
+ * partition_tokens : 0 = the built-in choice (see pa_decode); -1 = the
+ *                    balanced schedule whatever the work (batch <= 4096,
+ *                    else PA_ERR_UNSUPPORTED); > 0 = one CTA per (request,
+ *                    KV head, partition of this many tokens, a multiple of
+ *                    block_size).  The workspace must be sized with
+ *                    pa_decode_workspace_size_ex for the same value. */
+/* *balanced_out (may be NULL): 1 when the call uses the balanced schedule. */
 int pa_decode_workspace_size_ex(int batch, int num_q_heads, int num_kv_heads, int head_dim,
                                 int block_size, int max_seq_len, int partition_tokens,
-                                size_t* bytes_out, int* num_partitions_out);
+                                size_t* bytes_out, int* num_partitions_out, int* balanced_out);
 
 int pa_decode_ex(pa_bf16* out, const pa_bf16* q, const pa_bf16* kv_pool,
                  const int32_t* block_tables, const int32_t* seq_lens, int batch,

@@ -40,6 +40,8 @@ PA_DECODE_AUTO = 0
 PA_DECODE_CUDA_CORE = 1
 PA_DECODE_MMA = 2
 
+PA_SCHEDULE_BALANCED = -1  # partition_tokens value that asks for the balanced schedule
+
 _c = ctypes
 _P = _c.c_void_p
 _I = _c.c_int
@@ -54,7 +56,7 @@ _SIGNATURES = {
     "pa_reshape_and_cache": (_I, [_P, _P, _P, _P, _I, _I, _I, _I, _I, _P]),
     "pa_copy_blocks": (_I, [_P, _P, _I, _I, _I, _I, _I, _P]),
     "pa_decode_workspace_size": (_I, [_I, _I, _I, _I, _I, _I, _P, _P]),
-    "pa_decode_workspace_size_ex": (_I, [_I, _I, _I, _I, _I, _I, _I, _P, _P]),
+    "pa_decode_workspace_size_ex": (_I, [_I, _I, _I, _I, _I, _I, _I, _P, _P, _P]),
     "pa_decode": (_I, [_P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _I, _I, _c.c_float, _P, _SZ, _P]),
     "pa_decode_ex": (_I, [_P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _I, _I, _c.c_float, _P, _SZ,
                           _I, _I, _P]),
@@ -176,13 +178,18 @@ def pa_copy_blocks(kv_pool, block_pairs, stream=None):
 
 
 def pa_decode_workspace_size(batch, num_q_heads, num_kv_heads, head_dim, block_size, max_seq_len,
-                             partition_tokens=0):
-    """(bytes, num_partitions) of the split-K scratch pa_decode needs."""
+                             partition_tokens=0, with_schedule=False):
+    """(bytes, num_partitions) of the split-K scratch pa_decode needs; with
+    ``with_schedule`` also "balanced" or "grid"."""
     nbytes = ctypes.c_size_t(0)
     parts = ctypes.c_int(0)
+    balanced = ctypes.c_int(0)
     _check(lib.pa_decode_workspace_size_ex(batch, num_q_heads, num_kv_heads, head_dim, block_size,
                                            max_seq_len, partition_tokens, ctypes.byref(nbytes),
-                                           ctypes.byref(parts)), "pa_decode_workspace_size")
+                                           ctypes.byref(parts), ctypes.byref(balanced)),
+           "pa_decode_workspace_size")
+    if with_schedule:
+        return nbytes.value, parts.value, ("balanced" if balanced.value else "grid")
     return nbytes.value, parts.value
 
 

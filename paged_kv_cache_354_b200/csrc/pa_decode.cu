@@ -1155,15 +1155,23 @@ struct Plan {
 
 static size_t align256(size_t x) { return (x + 255) & ~static_cast<size_t>(255); }
 
-// partition_tokens == 0 selects the balanced schedule (batches up to
-// kStreamMaxBatch); a positive value selects the per-partition grid with
+// partition_tokens: 0 = choose (balanced when the batch fits and has enough
+// work), kForceBalanced = balanced, > 0 = per-partition grid with
 // partitions of that many tokens.
+constexpr int kForceBalanced = -1;
 static int make_plan(int batch, int hq, int hkv, int d, int bs, int max_seq_len,
                      int partition_tokens, Plan* plan) {
   const int nblk_max = max_seq_len > 0 ? (max_seq_len + bs - 1) / bs : 1;
   const int group = hq / hkv;
-  if (partition_tokens == 0 && batch <= kStreamMaxBatch) {
-    const int sms = sm_count() > 0 ? sm_count() : 148;
+  const int sms = sm_count() > 0 ? sm_count() : 148;
+  // the balanced schedule pays when there are at least a few blocks per
+  // persistent CTA; tiny batches (launch-bound anyway) take the grid
+  const long long units_max = static_cast<long long>(batch) * hkv * nblk_max;
+  if (partition_tokens == kForceBalanced && batch > kStreamMaxBatch)
+    return fail(PA_ERR_UNSUPPORTED, "balanced schedule: batch %d above %d", batch, kStreamMaxBatch);
+  if (partition_tokens == kForceBalanced ||
+      (partition_tokens == 0 && batch <= kStreamMaxBatch &&
+       units_max >= 2ll * sms * kStreamCtasPerSm)) {
     plan->stream = true;
     plan->ctas = sms * kStreamCtasPerSm;
     plan->part_blocks = 1;  // set per call from max_blocks_per_seq
@@ -1182,10 +1190,9 @@ static int make_plan(int batch, int hq, int hkv, int d, int bs, int max_seq_len,
                   partition_tokens, bs);
     pb = partition_tokens / bs;
   } else {
-    // batches above the stream limit: 512-token partitions, halved while the
-    // grid would leave the SMs short of work
+    // batches above the stream limit, or too little work for it: 512-token
+    // partitions, halved while the grid would leave the SMs short of work
     pb = 512 / bs;
-    const int sms = sm_count() > 0 ? sm_count() : 148;
     const long long pairs = static_cast<long long>(batch) * hkv;
     while (pb > 4 && pairs * ((nblk_max + pb - 1) / pb) < 4ll * sms) pb /= 2;
   }
@@ -1290,7 +1297,8 @@ static int decode_impl(pa_bf16* out, const pa_bf16* q, const pa_bf16* kv_pool,
   if (rc != PA_OK) return rc;
   if (num_blocks <= 0 || max_blocks <= 0)
     return fail(PA_ERR_INVALID, "pa_decode: num_blocks and max_blocks_per_seq must be positive");
-  if (partition_tokens < 0) return fail(PA_ERR_INVALID, "pa_decode: negative partition_tokens");
+  if (partition_tokens < kForceBalanced)
+    return fail(PA_ERR_INVALID, "pa_decode: partition_tokens %d below -1", partition_tokens);
   if (!std::isfinite(scale)) return fail(PA_ERR_INVALID, "pa_decode: scale is not finite");
   if (batch == 0) return PA_OK;
   if (!out || !q || !kv_pool || !block_tables || !seq_lens)
@@ -1363,18 +1371,20 @@ extern "C" {
 
 int pa_decode_workspace_size_ex(int batch, int num_q_heads, int num_kv_heads, int head_dim,
                                 int block_size, int max_seq_len, int partition_tokens,
-                                size_t* bytes_out, int* num_partitions_out) {
+                                size_t* bytes_out, int* num_partitions_out, int* balanced_out) {
   using namespace pa;
   if (bytes_out == nullptr) return fail(PA_ERR_INVALID, "pa_decode_workspace_size: NULL bytes_out");
   int rc = check_shape(batch, num_q_heads, num_kv_heads, head_dim, block_size, max_seq_len);
   if (rc != PA_OK) return rc;
-  if (partition_tokens < 0) return fail(PA_ERR_INVALID, "negative partition_tokens");
+  if (partition_tokens < kForceBalanced)
+    return fail(PA_ERR_INVALID, "partition_tokens %d below -1", partition_tokens);
   Plan plan;
   rc = make_plan(batch, num_q_heads, num_kv_heads, head_dim, block_size, max_seq_len,
                  partition_tokens, &plan);
   if (rc != PA_OK) return rc;
   *bytes_out = plan.bytes;
   if (num_partitions_out) *num_partitions_out = plan.stream ? plan.ctas : plan.max_parts;
+  if (balanced_out) *balanced_out = plan.stream ? 1 : 0;
   return PA_OK;
 }
 
@@ -1382,7 +1392,7 @@ int pa_decode_workspace_size(int batch, int num_q_heads, int num_kv_heads, int h
                              int block_size, int max_seq_len, size_t* bytes_out,
                              int* num_partitions_out) {
   return pa_decode_workspace_size_ex(batch, num_q_heads, num_kv_heads, head_dim, block_size,
-                                     max_seq_len, 0, bytes_out, num_partitions_out);
+                                     max_seq_len, 0, bytes_out, num_partitions_out, nullptr);
 }
 
 int pa_decode(pa_bf16* out, const pa_bf16* q, const pa_bf16* kv_pool, const int32_t* block_tables,

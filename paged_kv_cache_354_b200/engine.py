@@ -44,9 +44,9 @@ class PagedDecodeCache:
         self.pool = torch.empty((self.num_blocks, 2, num_kv_heads, block_size, head_dim),
                                 dtype=torch.bfloat16, device=self.device)
         self.alloc = PaAlloc(self.num_blocks, block_size, initial_order)
-        nbytes, self.num_partitions = pa_decode_workspace_size(
+        nbytes, self.num_partitions, self.schedule = pa_decode_workspace_size(
             self.max_batch, num_q_heads, num_kv_heads, head_dim, block_size, self.max_seq_len,
-            partition_tokens)
+            partition_tokens, with_schedule=True)
         self.workspace = torch.empty(max(nbytes, 256), dtype=torch.uint8, device=self.device)
         # one pinned buffer (and its device twin) for a step's metadata:
         # slots int64[B] | lens int32[B] | pairs int32[B,2] | tables int32[B,MB]

@@ -67,7 +67,12 @@ def test_invalid_arguments_fail_before_launch():
         pk.PA_ERR_INVALID
     # partition size must be a whole number of blocks
     assert lib.pa_decode_workspace_size_ex(4, 8, 2, 128, 16, 1000, 100, ctypes.byref(nb),
-                                           ctypes.byref(parts)) == pk.PA_ERR_INVALID
+                                           ctypes.byref(parts), None) == pk.PA_ERR_INVALID
+    # the balanced schedule on request only up to its batch limit; -2 is no schedule
+    assert lib.pa_decode_workspace_size_ex(5000, 8, 2, 128, 16, 1000, -1, ctypes.byref(nb),
+                                           ctypes.byref(parts), None) == pk.PA_ERR_UNSUPPORTED
+    assert lib.pa_decode_workspace_size_ex(4, 8, 2, 128, 16, 1000, -2, ctypes.byref(nb),
+                                           ctypes.byref(parts), None) == pk.PA_ERR_INVALID
     # batch 0 decode is a no-op
     assert lib.pa_decode(None, None, None, None, None, 0, 8, 2, 128, 16, 10, 4, 0, 1.0, None, 0, None) == pk.PA_OK
     assert lib.pa_selftest_wait_timeout(0, None) == pk.PA_ERR_INVALID
@@ -75,8 +80,9 @@ def test_invalid_arguments_fail_before_launch():
 
 def test_explicit_partition_sizes_workspace():
     # explicit partitions do not consult the device
-    nbytes, parts = pk.pa_decode_workspace_size(2, 8, 2, 128, 16, 1000, partition_tokens=256)
-    assert parts == 4
+    nbytes, parts, sched = pk.pa_decode_workspace_size(2, 8, 2, 128, 16, 1000, partition_tokens=256,
+                                                       with_schedule=True)
+    assert parts == 4 and sched == "grid"
     rows = 2 * 8 * 4
     assert nbytes >= rows * 128 * 4 + 2 * rows * 4
     nbytes, parts = pk.pa_decode_workspace_size(2, 8, 2, 128, 16, 200, partition_tokens=256)

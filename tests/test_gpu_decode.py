@@ -56,8 +56,10 @@ def test_auto_variant_ragged(d, bs, group):
                                            ("mma", 1), ("mma", 2), ("mma", 3), ("mma", 4), ("mma", 5),
                                            ("mma", 8)])
 @pytest.mark.parametrize("d,bs", [(128, 16), (64, 32)])
-def test_each_variant(variant, group, d, bs):
-    check([5, 31, 33, 200, 480], 2 * group, 2, d, bs, seed=100 + group, variant=variant)
+@pytest.mark.parametrize("schedule", [pk.PA_SCHEDULE_BALANCED, 0, 64])
+def test_each_variant(variant, group, d, bs, schedule):
+    check([5, 31, 33, 200, 480], 2 * group, 2, d, bs, seed=100 + group, variant=variant,
+          partition_tokens=schedule)
 
 
 @pytest.mark.parametrize("partition_blocks", [1, 2, 3, 8, 64])
@@ -78,14 +80,14 @@ def test_split_k_partitions(partition_blocks, variant):
 @pytest.mark.parametrize("variant", ["mma", "cuda_core"])
 def test_balanced_schedule_edges(lens, variant):
     check(lens, 8 if variant == "mma" else 4, 2 if variant == "mma" else 4, 64, 16, seed=60 + len(lens),
-          variant=variant)
+          variant=variant, partition_tokens=pk.PA_SCHEDULE_BALANCED)
 
 
 def test_balanced_matches_partition_grid():
     lens = [3000, 17, 1200, 2049, 5, 640, 2999, 1, 4096, 33]
     q, pool, _, (t, l) = make_case(lens, 32, 8, 128, 16, seed=61)
     q, pool = q.cuda(), pool.cuda()
-    bal = run_decode(q, pool, t, l, 0.088, pk.PA_DECODE_MMA, partition_tokens=0)
+    bal = run_decode(q, pool, t, l, 0.088, pk.PA_DECODE_MMA, partition_tokens=pk.PA_SCHEDULE_BALANCED)
     grid = run_decode(q, pool, t, l, 0.088, pk.PA_DECODE_MMA, partition_tokens=512)
     assert (bal.float() - grid.float()).abs().max().item() <= 2 ** -7
 
