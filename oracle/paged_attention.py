@@ -126,3 +126,31 @@ def decode_one(query_vec, kv_pool, block_table_row, seq_len, kv_head, scale):
     weights = np.exp(logits - logits.max())
     weights /= weights.sum()
     return weights @ values[:, kv_head, :]
+
+
+def decode_multi(query, kv_pool, block_tables, seq_lens, scale):
+    """T query tokens per request, each attending causally (float64).
+
+    The T newest tokens of request b are its queries: token t sits at
+    position L_b - T + t (its keys and values are already in the cache) and
+    attends to positions [0, L_b - T + t] -- the same gather and softmax as
+    ``decode`` over a prefix of the request.  This is the multi-token form a
+    speculative-verification or chunked decode step needs; the pages give
+    the single-token form, and a query token with no position to attend to
+    (L_b - T + t < 0) gets 0 like an empty request.
+
+    query : float64 [B, T, Hq, D]; returns float64 [B, T, Hq, D].
+    """
+    batch, tokens, num_q_heads, head_dim = query.shape
+    num_kv_heads = kv_pool.shape[2]
+    group = num_q_heads // num_kv_heads
+    out = np.zeros((batch, tokens, num_q_heads, head_dim), dtype=np.float64)
+    for b in range(batch):
+        for t in range(tokens):
+            visible = int(seq_lens[b]) - tokens + t + 1
+            if visible <= 0:
+                continue
+            for j in range(num_q_heads):
+                out[b, t, j] = decode_one(query[b, t, j], kv_pool, block_tables[b], visible,
+                                          j // group, scale)
+    return out

@@ -180,6 +180,56 @@ def pin_decode_one(m):
             np.testing.assert_allclose(one, full[i, j], rtol=0, atol=1e-14)
 
 
+def pin_multi_reduces_to_decode(m):
+    """T = 1 is exactly the single-token decode; token t of T equals a
+    single-token decode over the first L - T + t + 1 positions."""
+    rng = np.random.default_rng(12)
+    lens = [9, 21, 3]
+    q, ks, vs, pool, table = random_case(rng, lens, 4, 2, 8, 4)
+    one = m.decode_multi(q[:, None], pool, table, np.array(lens), 0.4)
+    np.testing.assert_array_equal(one[:, 0], m.decode(q, pool, table, np.array(lens), 0.4))
+    T = 4
+    qm = rng.standard_normal((3, T, 4, 8))
+    got = m.decode_multi(qm, pool, table, np.array(lens), 0.4)
+    for b, n in enumerate(lens):
+        for t in range(T):
+            vis = n - T + t + 1
+            want = m.decode(qm[b:b + 1, t], pool, table[b:b + 1], np.array([max(vis, 0)]), 0.4)
+            np.testing.assert_array_equal(got[b, t], want[0])
+
+
+def pin_multi_causal_sdpa(m):
+    """Against torch SDPA (fp64) with an explicit causal mask on contiguous K/V."""
+    rng = np.random.default_rng(13)
+    lens, T, hq, hkv, d = [7, 30, 16], 5, 8, 2, 16
+    ks = [rng.standard_normal((n, hkv, d)) for n in lens]
+    vs = [rng.standard_normal((n, hkv, d)) for n in lens]
+    pool, table = place_requests(ks, vs, 4, 20, rng)
+    q = rng.standard_normal((len(lens), T, hq, d))
+    got = m.decode_multi(q, pool, table, np.array(lens), 0.3)
+    for b, n in enumerate(lens):
+        g = hq // hkv
+        kt = torch.from_numpy(ks[b]).permute(1, 0, 2).repeat_interleave(g, dim=0)[None]
+        vt = torch.from_numpy(vs[b]).permute(1, 0, 2).repeat_interleave(g, dim=0)[None]
+        qt = torch.from_numpy(q[b]).permute(1, 0, 2)[None]  # [1, Hq, T, D]
+        pos = torch.arange(n)[None, :]
+        qpos = (n - T + torch.arange(T))[:, None]
+        mask = pos <= qpos  # [T, n]
+        ref = torch.nn.functional.scaled_dot_product_attention(qt, kt, vt, attn_mask=mask, scale=0.3)
+        ref = ref[0].permute(1, 0, 2).numpy()
+        np.testing.assert_allclose(got[b], ref, rtol=0, atol=1e-12)
+
+
+def pin_multi_short_request(m):
+    """Query tokens before the request's start attend to nothing: output 0."""
+    rng = np.random.default_rng(14)
+    q, ks, vs, pool, table = random_case(rng, [2], 2, 1, 8, 4)
+    qm = rng.standard_normal((1, 4, 2, 8))
+    got = m.decode_multi(qm, pool, table, np.array([2]), 0.5)
+    assert np.array_equal(got[0, :2], np.zeros((2, 2, 8)))
+    np.testing.assert_allclose(got[0, 3], m.decode(qm[:, 3], pool, table, np.array([2]), 0.5)[0], atol=0)
+
+
 DECODE_PINS = [
     pin_gather_is_contiguous,
     pin_sdpa,
@@ -190,6 +240,9 @@ DECODE_PINS = [
     pin_block_permutation_invariance,
     pin_empty_request,
     pin_decode_one,
+    pin_multi_reduces_to_decode,
+    pin_multi_causal_sdpa,
+    pin_multi_short_request,
 ]
 
 
@@ -212,6 +265,8 @@ MUTATIONS = {
     "not_normalised": ("            weights /= weights.sum()\n            out[b, j]", "            out[b, j]"),
     "keys_for_values": ("out[b, j] = weights @ values[:, h, :]", "out[b, j] = weights @ keys[:, h, :]"),
     "off_by_one_length": ("pos = np.arange(seq_len)", "pos = np.arange(1, seq_len + 1)"),
+    "multi_not_causal": ("visible = int(seq_lens[b]) - tokens + t + 1", "visible = int(seq_lens[b])"),
+    "multi_off_by_one": ("visible = int(seq_lens[b]) - tokens + t + 1", "visible = int(seq_lens[b]) - tokens + t"),
 }
 
 
