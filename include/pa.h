@@ -234,6 +234,32 @@ int pa_decode_noalloc(pa_bf16* out, const pa_bf16* q, const pa_bf16* kv_pool,
                       int num_blocks, int max_blocks_per_seq, int max_seq_len, float scale,
                       void* stream);
 
+/* --------------------------------------------------------------------------
+ * pa_decode_multi -- several query tokens per request, causal.
+ *
+ * The single-token operation above, for the T newest tokens of each request
+ * at once (speculative-decoding verification, chunked decode): query token
+ * t of request b sits at position seq_lens[b] - T + t -- its keys and values
+ * are already in the cache -- and attends to positions [0, seq_lens[b] - T
+ * + t] through the block table, as in the quiz page's sketch over that
+ * prefix.  A token with no position to attend to (seq_lens[b] < T - t) gets
+ * out = 0.
+ *
+ * q, out       : device bf16 [batch][T][num_q_heads][head_dim]
+ * Other arguments as pa_decode.  (num_q_heads / num_kv_heads) * T <= 16.
+ * Always the balanced schedule (batch <= 4096) and the tensor-core
+ * consumer; workspace from pa_decode_multi_workspace_size.
+ * ------------------------------------------------------------------------ */
+int pa_decode_multi_workspace_size(int batch, int num_query_tokens, int num_q_heads,
+                                   int num_kv_heads, int head_dim, int block_size,
+                                   int max_seq_len, size_t* bytes_out);
+
+int pa_decode_multi(pa_bf16* out, const pa_bf16* q, const pa_bf16* kv_pool,
+                    const int32_t* block_tables, const int32_t* seq_lens, int batch,
+                    int num_query_tokens, int num_q_heads, int num_kv_heads, int head_dim,
+                    int block_size, int num_blocks, int max_blocks_per_seq, int max_seq_len,
+                    float scale, void* workspace, size_t workspace_bytes, void* stream);
+
 /* Self-test of the bounded pipeline wait used by the kernels: one CTA waits
  * on a barrier phase that nothing completes, for at most limit_ns, then
  * returns.  Expect PA_DEVERR_WAIT_TIMEOUT in pa_device_error() afterwards.

@@ -61,6 +61,9 @@ _SIGNATURES = {
     "pa_decode_ex": (_I, [_P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _I, _I, _c.c_float, _P, _SZ,
                           _I, _I, _P]),
     "pa_decode_noalloc": (_I, [_P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _I, _I, _c.c_float, _P]),
+    "pa_decode_multi_workspace_size": (_I, [_I, _I, _I, _I, _I, _I, _I, _P]),
+    "pa_decode_multi": (_I, [_P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _I, _I, _I, _c.c_float, _P, _SZ,
+                             _P]),
     "pa_selftest_wait_timeout": (_I, [_I64, _P]),
     "pa_alloc_create": (_I, [_I, _I, _P, _P]),
     "pa_alloc_destroy": (_I, [_P]),
@@ -214,6 +217,34 @@ def pa_decode(out, q, kv_pool, block_tables, seq_lens, max_seq_len, scale, works
     _check(lib.pa_decode_ex(_ptr(out), _ptr(q), _ptr(kv_pool), _ptr(block_tables), _ptr(seq_lens), b, hq,
                             hkv, d, bs, nb, block_tables.shape[1], int(max_seq_len), float(scale), ws_ptr,
                             ws_bytes, int(variant), int(partition_tokens), _stream(stream)), "pa_decode")
+
+
+def pa_decode_multi_workspace_size(batch, num_query_tokens, num_q_heads, num_kv_heads, head_dim, block_size,
+                                   max_seq_len):
+    nbytes = ctypes.c_size_t(0)
+    _check(lib.pa_decode_multi_workspace_size(batch, num_query_tokens, num_q_heads, num_kv_heads, head_dim,
+                                              block_size, max_seq_len, ctypes.byref(nbytes)),
+           "pa_decode_multi_workspace_size")
+    return nbytes.value
+
+
+def pa_decode_multi(out, q, kv_pool, block_tables, seq_lens, max_seq_len, scale, workspace, stream=None):
+    """T causal query tokens per request: q, out bf16 [B, T, Hq, D]."""
+    import torch
+
+    _require(out, torch.bfloat16, "out")
+    _require(q, torch.bfloat16, "q")
+    _require(kv_pool, torch.bfloat16, "kv_pool")
+    _require(block_tables, torch.int32, "block_tables")
+    _require(seq_lens, torch.int32, "seq_lens")
+    _require(workspace, torch.uint8, "workspace")
+    nb, two, hkv, bs, d = kv_pool.shape
+    b, t, hq, dq = q.shape
+    if out.shape != q.shape or dq != d or block_tables.shape[0] != b or seq_lens.shape != (b,):
+        raise ValueError("pa_decode_multi: shape mismatch")
+    _check(lib.pa_decode_multi(_ptr(out), _ptr(q), _ptr(kv_pool), _ptr(block_tables), _ptr(seq_lens), b, t, hq,
+                               hkv, d, bs, nb, block_tables.shape[1], int(max_seq_len), float(scale),
+                               _ptr(workspace), workspace.numel(), _stream(stream)), "pa_decode_multi")
 
 
 PA_NOALLOC_SCRATCH_BYTES = 16 * 1024 * 1024

@@ -89,6 +89,8 @@ struct DecodeArgs {
   int part_blocks, max_parts;
   float scale_log2;  // scale * log2(e)
   int* stream_prefix;  // balanced schedule: per-request block-count prefix sums [B+1]
+  int qtok;            // query tokens per request (1 = single-token decode)
+  int cols;            // group * qtok: (token, head) columns per KV head
 };
 
 // Tokens of request b the kernels attend over, after the device-side checks
@@ -107,44 +109,60 @@ __device__ __forceinline__ int effective_len(int raw, int bs, const DecodeArgs& 
 
 // --------------------------------------------------------------------------
 // Tensor-core consumer: state and per-block step.
+//
+// The 8*NT columns of S^T are (query token, query head) pairs: column
+// c = t * g + j is head j of the KV head's group for query token t, which
+// may attend to positions <= lim(c) = len - T + t (T = 1: the whole request).
+// Columns past g * T are padding (zero query, never stored).
 // --------------------------------------------------------------------------
-template <int D, int BS>
+template <int D, int BS, int NT>
 struct MmaConsumer {
   using geo = Geo<D, BS>;
   static constexpr int kDT = D / 16;   // 16-dim tiles of the head dim
   static constexpr int kTT = BS / 16;  // 16-token tiles of a block
-  uint32_t qb[kDT][2];                 // Q^T as the B operand of S^T = K Q^T
-  float o[kDT][4];                     // O^T accumulators
-  float m0, m1, l0, l1;                // two head columns of this thread
+  uint32_t qb[NT][kDT][2];             // Q^T as the B operand of S^T = K Q^T
+  float o[kDT][NT][4];                 // O^T accumulators
+  float m[NT][2], l[NT][2];            // two columns per n-tile of this thread
+  int lim[NT][2];                      // last position each of those columns sees
 
-  __device__ __forceinline__ void init(const __nv_bfloat16* qrow_base, int group, int lane) {
-    const int head = lane >> 2;
+  // qbase: Q row of (token 0, head 0) of this KV head's group; consecutive
+  // tokens are q_tok_stride elements apart, heads D apart.
+  __device__ __forceinline__ void init(const __nv_bfloat16* qbase, int cols, int group, int qtok,
+                                       size_t q_tok_stride, int len, int lane) {
     const int c = 2 * (lane & 3);
 #pragma unroll
-    for (int ks = 0; ks < kDT; ++ks) {
-      if (head < group) {
-        const __nv_bfloat16* qr = qrow_base + head * D + 16 * ks + c;
-        qb[ks][0] = *reinterpret_cast<const uint32_t*>(qr);
-        qb[ks][1] = *reinterpret_cast<const uint32_t*>(qr + 8);
-      } else {
-        qb[ks][0] = 0u;
-        qb[ks][1] = 0u;
-      }
-    }
+    for (int nt = 0; nt < NT; ++nt) {
+      const int col = nt * 8 + (lane >> 2);  // B-operand column of this thread
+      const bool real = col < cols;
+      const int t = real ? col / group : 0;
+      const __nv_bfloat16* qr = qbase + t * q_tok_stride + (col - t * group) * D + c;
 #pragma unroll
-    for (int dt = 0; dt < kDT; ++dt) o[dt][0] = o[dt][1] = o[dt][2] = o[dt][3] = 0.f;
-    m0 = m1 = -INFINITY;
-    l0 = l1 = 0.f;
+      for (int ks = 0; ks < kDT; ++ks) {
+        qb[nt][ks][0] = real ? *reinterpret_cast<const uint32_t*>(qr + 16 * ks) : 0u;
+        qb[nt][ks][1] = real ? *reinterpret_cast<const uint32_t*>(qr + 16 * ks + 8) : 0u;
+      }
+#pragma unroll
+      for (int e = 0; e < 2; ++e) {
+        const int cc = nt * 8 + c + e;  // accumulator column of this thread
+        lim[nt][e] = cc < cols ? len - qtok + cc / group : len - 1;
+        m[nt][e] = -INFINITY;
+        l[nt][e] = 0.f;
+      }
+#pragma unroll
+      for (int dt = 0; dt < kDT; ++dt) o[dt][nt][0] = o[dt][nt][1] = o[dt][nt][2] = o[dt][nt][3] = 0.f;
+    }
   }
 
-  __device__ __forceinline__ void step(uint32_t sb, int valid, float scale_log2, int lane) {
+  // sb: staged block; pos0: position of its row 0 in the request.
+  __device__ __forceinline__ void step(uint32_t sb, int pos0, float scale_log2, int lane) {
     const int mat = lane >> 3;
     const int r8 = lane & 7;
-    // ---- S^T = K Q^T : rows = tokens, cols = query heads of the group
-    float s[kTT][4];
+    // ---- S^T = K Q^T : rows = tokens of the block, cols = (token, head)
+    float s[kTT][NT][4];
 #pragma unroll
     for (int mt = 0; mt < kTT; ++mt) {
-      s[mt][0] = s[mt][1] = s[mt][2] = s[mt][3] = 0.f;
+#pragma unroll
+      for (int nt = 0; nt < NT; ++nt) s[mt][nt][0] = s[mt][nt][1] = s[mt][nt][2] = s[mt][nt][3] = 0.f;
       const int tok = 16 * mt + ((mat & 1) << 3) + r8;
 #pragma unroll
       for (int ks = 0; ks < kDT; ++ks) {
@@ -152,53 +170,73 @@ struct MmaConsumer {
         const uint32_t addr = sb + (ks >> 2) * geo::kRegionBytes + tok * 128 + chunk * 16;
         uint32_t a0, a1, a2, a3;
         ldsm_x4(addr, a0, a1, a2, a3);
-        mma_bf16_16816(s[mt], a0, a1, a2, a3, qb[ks][0], qb[ks][1]);
+#pragma unroll
+        for (int nt = 0; nt < NT; ++nt) mma_bf16_16816(s[mt][nt], a0, a1, a2, a3, qb[nt][ks][0], qb[nt][ks][1]);
       }
     }
-    // ---- scale, mask rows past the request's end, column max
-    float mx0 = -INFINITY, mx1 = -INFINITY;
+    // ---- scale, mask positions each column may not see, column max
+    float mx[NT][2];
+#pragma unroll
+    for (int nt = 0; nt < NT; ++nt) mx[nt][0] = mx[nt][1] = -INFINITY;
 #pragma unroll
     for (int mt = 0; mt < kTT; ++mt) {
-      const int t0 = 16 * mt + (lane >> 2);
-      const bool ok0 = t0 < valid, ok1 = t0 + 8 < valid;
-      s[mt][0] = ok0 ? s[mt][0] * scale_log2 : -INFINITY;
-      s[mt][1] = ok0 ? s[mt][1] * scale_log2 : -INFINITY;
-      s[mt][2] = ok1 ? s[mt][2] * scale_log2 : -INFINITY;
-      s[mt][3] = ok1 ? s[mt][3] * scale_log2 : -INFINITY;
-      mx0 = fmaxf(mx0, fmaxf(s[mt][0], s[mt][2]));
-      mx1 = fmaxf(mx1, fmaxf(s[mt][1], s[mt][3]));
-    }
+      const int p0 = pos0 + 16 * mt + (lane >> 2);
 #pragma unroll
-    for (int off = 4; off < 32; off <<= 1) {
-      mx0 = fmaxf(mx0, __shfl_xor_sync(kFull, mx0, off));
-      mx1 = fmaxf(mx1, __shfl_xor_sync(kFull, mx1, off));
+      for (int nt = 0; nt < NT; ++nt) {
+#pragma unroll
+        for (int e = 0; e < 2; ++e) {
+          s[mt][nt][e] = p0 <= lim[nt][e] ? s[mt][nt][e] * scale_log2 : -INFINITY;
+          s[mt][nt][e + 2] = p0 + 8 <= lim[nt][e] ? s[mt][nt][e + 2] * scale_log2 : -INFINITY;
+          mx[nt][e] = fmaxf(mx[nt][e], fmaxf(s[mt][nt][e], s[mt][nt][e + 2]));
+        }
+      }
     }
-    const float n0 = fmaxf(m0, mx0), n1 = fmaxf(m1, mx1);
+    bool moved = false;
+#pragma unroll
+    for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+      for (int e = 0; e < 2; ++e) {
+#pragma unroll
+        for (int off = 4; off < 32; off <<= 1)
+          mx[nt][e] = fmaxf(mx[nt][e], __shfl_xor_sync(kFull, mx[nt][e], off));
+        mx[nt][e] = fmaxf(m[nt][e], mx[nt][e]);
+        moved |= mx[nt][e] > m[nt][e];
+      }
     // rescale only when some column's running max moved (warp-uniform test)
-    if (__any_sync(kFull, (n0 > m0) || (n1 > m1))) {
-      const float a0 = (m0 == -INFINITY) ? 0.f : exp2f(m0 - n0);
-      const float a1 = (m1 == -INFINITY) ? 0.f : exp2f(m1 - n1);
+    if (__any_sync(kFull, moved)) {
 #pragma unroll
-      for (int dt = 0; dt < kDT; ++dt) {
-        o[dt][0] *= a0;
-        o[dt][2] *= a0;
-        o[dt][1] *= a1;
-        o[dt][3] *= a1;
-      }
-      l0 *= a0;
-      l1 *= a1;
-      m0 = n0;
-      m1 = n1;
+      for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+        for (int e = 0; e < 2; ++e) {
+          const float a = (m[nt][e] == -INFINITY) ? 0.f : exp2f(m[nt][e] - mx[nt][e]);
+#pragma unroll
+          for (int dt = 0; dt < kDT; ++dt) {
+            o[dt][nt][e] *= a;
+            o[dt][nt][e + 2] *= a;
+          }
+          l[nt][e] *= a;
+          m[nt][e] = mx[nt][e];
+        }
     }
-    // ---- P (bf16) -> P^T fragments; O^T += V^T P^T
+    // ---- P (bf16) -> P^T fragments; O^T += V^T P^T.  A column that has seen
+    // no visible position yet keeps m = -inf: its p must be 0, not NaN.
+    float msafe[NT][2];
+#pragma unroll
+    for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+      for (int e = 0; e < 2; ++e) msafe[nt][e] = m[nt][e] == -INFINITY ? 0.f : m[nt][e];
 #pragma unroll
     for (int mt = 0; mt < kTT; ++mt) {
-      const uint32_t pa = pack_bf16x2(exp2f(s[mt][0] - m0), exp2f(s[mt][1] - m1));
-      const uint32_t pb = pack_bf16x2(exp2f(s[mt][2] - m0), exp2f(s[mt][3] - m1));
-      l0 += bf16lo_to_f32(pa) + bf16lo_to_f32(pb);
-      l1 += bf16hi_to_f32(pa) + bf16hi_to_f32(pb);
-      const uint32_t b0 = movmatrix_trans(pa);
-      const uint32_t b1 = movmatrix_trans(pb);
+      uint32_t b0[NT], b1[NT];
+#pragma unroll
+      for (int nt = 0; nt < NT; ++nt) {
+        const uint32_t pa = pack_bf16x2(exp2f(s[mt][nt][0] - msafe[nt][0]), exp2f(s[mt][nt][1] - msafe[nt][1]));
+        const uint32_t pb = pack_bf16x2(exp2f(s[mt][nt][2] - msafe[nt][0]), exp2f(s[mt][nt][3] - msafe[nt][1]));
+        l[nt][0] += bf16lo_to_f32(pa) + bf16lo_to_f32(pb);
+        l[nt][1] += bf16hi_to_f32(pa) + bf16hi_to_f32(pb);
+        b0[nt] = movmatrix_trans(pa);
+        b1[nt] = movmatrix_trans(pb);
+      }
       const int row = BS + 16 * mt + ((mat >> 1) << 3) + r8;
 #pragma unroll
       for (int dt = 0; dt < kDT; ++dt) {
@@ -206,34 +244,41 @@ struct MmaConsumer {
         const uint32_t addr = sb + (dt >> 2) * geo::kRegionBytes + row * 128 + chunk * 16;
         uint32_t a0, a1, a2, a3;
         ldsm_x4_trans(addr, a0, a1, a2, a3);
-        mma_bf16_16816(o[dt], a0, a1, a2, a3, b0, b1);
+#pragma unroll
+        for (int nt = 0; nt < NT; ++nt) mma_bf16_16816(o[dt][nt], a0, a1, a2, a3, b0[nt], b1[nt]);
       }
     }
   }
 
   // Write this warp's unnormalised O, running max and sum to the epilogue
-  // scratch: o_s[head][dim] (row stride kOStride), m_s[head], l_s[head].
+  // scratch: o_s[column][dim] (row stride kOStride), m_s[column], l_s[column].
   __device__ __forceinline__ void store(float* o_s, float* m_s, float* l_s, int lane) {
+    const int c = 2 * (lane & 3);
 #pragma unroll
-    for (int off = 4; off < 32; off <<= 1) {
-      l0 += __shfl_xor_sync(kFull, l0, off);
-      l1 += __shfl_xor_sync(kFull, l1, off);
-    }
-    const int h0 = 2 * (lane & 3);
+    for (int nt = 0; nt < NT; ++nt) {
 #pragma unroll
-    for (int dt = 0; dt < kDT; ++dt) {
-      const int d = 16 * dt + (lane >> 2);
-      constexpr int S = geo::kOStride;
-      o_s[h0 * S + d] = o[dt][0];
-      o_s[(h0 + 1) * S + d] = o[dt][1];
-      o_s[h0 * S + d + 8] = o[dt][2];
-      o_s[(h0 + 1) * S + d + 8] = o[dt][3];
-    }
-    if (lane < 4) {
-      m_s[h0] = m0;
-      m_s[h0 + 1] = m1;
-      l_s[h0] = l0;
-      l_s[h0 + 1] = l1;
+      for (int e = 0; e < 2; ++e) {
+        float le = l[nt][e];
+#pragma unroll
+        for (int off = 4; off < 32; off <<= 1) le += __shfl_xor_sync(kFull, le, off);
+        l[nt][e] = le;
+      }
+      const int c0 = nt * 8 + c;
+#pragma unroll
+      for (int dt = 0; dt < kDT; ++dt) {
+        const int d = 16 * dt + (lane >> 2);
+        constexpr int S = geo::kOStride;
+        o_s[c0 * S + d] = o[dt][nt][0];
+        o_s[(c0 + 1) * S + d] = o[dt][nt][1];
+        o_s[c0 * S + d + 8] = o[dt][nt][2];
+        o_s[(c0 + 1) * S + d + 8] = o[dt][nt][3];
+      }
+      if (lane < 4) {
+        m_s[c0] = m[nt][0];
+        m_s[c0 + 1] = m[nt][1];
+        l_s[c0] = l[nt][0];
+        l_s[c0 + 1] = l[nt][1];
+      }
     }
   }
 };
@@ -399,11 +444,11 @@ struct CudaCoreConsumer {
 // --------------------------------------------------------------------------
 // One consumer warp's work on one staged block (shared by both schedules).
 // --------------------------------------------------------------------------
-template <int D, int BS, int VAR, int G>
-__device__ __forceinline__ void consume_block(MmaConsumer<D, BS>& mc,
+template <int D, int BS, int VAR, int G, int NT>
+__device__ __forceinline__ void consume_block(MmaConsumer<D, BS, NT>& mc,
                                               CudaCoreConsumer<D, BS, (G > 0 ? G : 1)>& cc,
-                                              uint32_t sb, float* pbuf, int valid, float scale_log2,
-                                              int lane) {
+                                              uint32_t sb, float* pbuf, int valid, int pos0,
+                                              float scale_log2, int lane) {
   using geo = Geo<D, BS>;
   if constexpr (VAR == kMma) {
     if (valid < BS) {
@@ -423,7 +468,7 @@ __device__ __forceinline__ void consume_block(MmaConsumer<D, BS>& mc,
       fence_proxy_async_smem();
       __syncwarp();
     }
-    mc.step(sb, valid, scale_log2, lane);
+    mc.step(sb, pos0, scale_log2, lane);
   } else {
     cc.step(sb, pbuf, valid, scale_log2, lane);
   }
@@ -483,7 +528,7 @@ __global__ void __launch_bounds__(kThreads, (VAR == kMma || G <= 2) ? 3 : 2)
   }
   __syncthreads();
 
-  [[maybe_unused]] MmaConsumer<D, BS> mc;
+  [[maybe_unused]] MmaConsumer<D, BS, 1> mc;
   [[maybe_unused]] CudaCoreConsumer<D, BS, (G > 0 ? G : 1)> cc;
   if (warp == kConsumerWarps) {
     // ------------------------------------------------------------ producer
@@ -532,8 +577,10 @@ __global__ void __launch_bounds__(kThreads, (VAR == kMma || G <= 2) ? 3 : 2)
     // ----------------------------------------------------------- consumers
     const __nv_bfloat16* qrow = a.q + head0 * D;
     float* pbuf = reinterpret_cast<float*>(smem + sm::kPbuf) + warp * BS * (G > 0 ? G : 1);
-    if constexpr (VAR == kMma) mc.init(qrow, g, lane);
-    else cc.init(qrow, lane);
+    if constexpr (VAR == kMma)
+      mc.init(qrow, g, g, 1, static_cast<size_t>(a.num_q_heads) * D, len, lane);
+    else
+      cc.init(qrow, lane);
     for (int i = warp; i < n; i += kConsumerWarps) {
       if (*abort_flag) break;
       const int s = i % geo::kStages;
@@ -546,7 +593,7 @@ __global__ void __launch_bounds__(kThreads, (VAR == kMma || G <= 2) ? 3 : 2)
       }
       const uint32_t sb = sbase + s * geo::kStageBytes;
       const int valid = (blk0 + i == nblk - 1) ? last_valid : BS;
-      consume_block<D, BS, VAR, G>(mc, cc, sb, pbuf, valid, a.scale_log2, lane);
+      consume_block<D, BS, VAR, G, 1>(mc, cc, sb, pbuf, valid, (blk0 + i) * BS, a.scale_log2, lane);
       __syncwarp();
       if (lane == 0) mbar_arrive(bar_empty + 8 * s);
     }
@@ -643,9 +690,10 @@ __global__ void __launch_bounds__(kThreads, (VAR == kMma || G <= 2) ? 3 : 2)
 constexpr int kStreamCtasPerSm = PA_STREAM_CTAS_PER_SM;
 constexpr int kStreamMaxBatch = 4096;  // the prefix table lives in shared memory
 
-template <int D, int BS, int G>
+template <int D, int BS, int G, int NT>
 struct StreamSmem {
   using geo = Geo<D, BS>;
+  static constexpr int kCols = 8 * NT;  // epilogue rows per warp: (token, head) columns
   // Stage s must always be consumed by warp s % kConsumerWarps: a warp then
   // takes a stage's rounds one after the other, so a parity wait (which
   // only tells the current phase from the previous one) never runs two
@@ -661,7 +709,8 @@ struct StreamSmem {
   static constexpr int kPbuf = kScan + (kThreads + 4) * 4;       // CUDA-core p tiles
   static constexpr int kPbufBytes = kConsumerWarps * BS * (G > 0 ? G : 1) * 4;
   static constexpr int kEpi = (kPbuf + kPbufBytes + 15) & ~15;   // per-warp O, m, l
-  static constexpr int kPrefix = kEpi + geo::kEpiBytes;          // int32 [batch + 1]
+  static constexpr int kEpiO = kConsumerWarps * kCols * geo::kOStride * 4;
+  static constexpr int kPrefix = kEpi + kEpiO + 2 * kConsumerWarps * kCols * 4;  // int32 [batch+1]
   static constexpr int dynamic_bytes(int batch) { return kPrefix + 4 * (batch + 1) + 1024; }
 };
 
@@ -759,12 +808,12 @@ __device__ __forceinline__ void consumer_bar() {
   asm volatile("bar.sync 1, %0;" ::"n"(kConsumerWarps * 32) : "memory");
 }
 
-template <int D, int BS, int VAR, int G>
+template <int D, int BS, int VAR, int G, int NT>
 __global__ void __launch_bounds__(kThreads, kStreamCtasPerSm)
     paged_decode_stream_kernel(const __grid_constant__ CUtensorMap kv_map, const DecodeArgs a,
                                int batch) {
   using geo = Geo<D, BS>;
-  using sm = StreamSmem<D, BS, G>;
+  using sm = StreamSmem<D, BS, G, NT>;
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw_base = smem_u32(smem_raw);
   const uint32_t pad = ((raw_base + 1023u) & ~1023u) - raw_base;
@@ -801,7 +850,7 @@ __global__ void __launch_bounds__(kThreads, kStreamCtasPerSm)
   const long long u_end = stream_begin(total, blockIdx.x + 1, ctas);
   if (u_begin >= u_end) return;  // uniform: this CTA has no units
 
-  [[maybe_unused]] MmaConsumer<D, BS> mc;
+  [[maybe_unused]] MmaConsumer<D, BS, NT> mc;
   [[maybe_unused]] CudaCoreConsumer<D, BS, (G > 0 ? G : 1)> cc;
   if (warp == kConsumerWarps) {
     // ------------------------------------------------------------ producer
@@ -857,9 +906,12 @@ __global__ void __launch_bounds__(kThreads, kStreamCtasPerSm)
   } else {
     // ----------------------------------------------------------- consumers
     float* pbuf = reinterpret_cast<float*>(smem + sm::kPbuf) + warp * BS * (G > 0 ? G : 1);
+    constexpr int kC = sm::kCols;
     float* o_all = reinterpret_cast<float*>(smem + sm::kEpi);
-    float* m_all = reinterpret_cast<float*>(smem + sm::kEpi + geo::kEpiO);
-    float* l_all = m_all + kConsumerWarps * kMaxGroup;
+    float* m_all = reinterpret_cast<float*>(smem + sm::kEpi + sm::kEpiO);
+    float* l_all = m_all + kConsumerWarps * kC;
+    const int cols = a.cols;
+    const size_t q_tok_stride = static_cast<size_t>(a.num_q_heads) * D;
     int b, h, k;
     stream_locate(prefix, batch, hkv, u_begin, b, h, k);
     long long u = u_begin;
@@ -869,12 +921,13 @@ __global__ void __launch_bounds__(kThreads, kStreamCtasPerSm)
       const int nb = prefix[b + 1] - prefix[b];
       const int cnt = static_cast<int>(min(static_cast<long long>(nb - k), u_end - u));
       const bool complete = (k == 0 && cnt == nb);
-      const size_t head0 = static_cast<size_t>(b) * a.num_q_heads + static_cast<size_t>(h) * g;
+      // Q row of (token 0, head 0) of this KV head's group; out rows alike
+      const size_t qrow0 = static_cast<size_t>(b) * a.qtok * a.num_q_heads + static_cast<size_t>(h) * g;
       const int len = effective_len(__ldg(a.seq_lens + b), BS, a, false);
       const int last_valid = len - (nb - 1) * BS;
-      const __nv_bfloat16* qrow = a.q + head0 * D;
-      if constexpr (VAR == kMma) mc.init(qrow, g, lane);
-      else cc.init(qrow, lane);
+      const __nv_bfloat16* qbase = a.q + qrow0 * D;
+      if constexpr (VAR == kMma) mc.init(qbase, cols, g, a.qtok, q_tok_stride, len, lane);
+      else cc.init(qbase, lane);
       // this warp's blocks of the segment: running indices i..i+cnt-1 that are
       // congruent to the warp number
       for (int ii = i + ((warp - i % kConsumerWarps + kConsumerWarps) % kConsumerWarps);
@@ -889,46 +942,49 @@ __global__ void __launch_bounds__(kThreads, kStreamCtasPerSm)
           break;
         }
         const uint32_t sb = sbase + s * geo::kStageBytes;
-        const int valid = (k + (ii - i) == nb - 1) ? last_valid : BS;
-        consume_block<D, BS, VAR, G>(mc, cc, sb, pbuf, valid, a.scale_log2, lane);
+        const int blk = k + (ii - i);
+        const int valid = (blk == nb - 1) ? last_valid : BS;
+        consume_block<D, BS, VAR, G, NT>(mc, cc, sb, pbuf, valid, blk * BS, a.scale_log2, lane);
         __syncwarp();
         if (lane == 0) mbar_arrive(bar_empty + 8 * s);
       }
       // ---- segment epilogue: merge the four warps' states
       {
-        float* o_s = o_all + warp * kMaxGroup * geo::kOStride;
-        if constexpr (VAR == kMma) mc.store(o_s, m_all + warp * kMaxGroup, l_all + warp * kMaxGroup, lane);
-        else cc.store(o_s, m_all + warp * kMaxGroup, l_all + warp * kMaxGroup, lane);
+        float* o_s = o_all + warp * kC * geo::kOStride;
+        if constexpr (VAR == kMma) mc.store(o_s, m_all + warp * kC, l_all + warp * kC, lane);
+        else cc.store(o_s, m_all + warp * kC, l_all + warp * kC, lane);
       }
       consumer_bar();
       if (*abort_flag == 0) {
         const int slot = (seg == 0) ? 0 : 1;
-        const size_t prow = (static_cast<size_t>(blockIdx.x) * 2 + slot) * g;
-        for (int idx = threadIdx.x; idx < g * D / 2; idx += kConsumerWarps * 32) {
-          const int j = (2 * idx) / D;
+        const size_t prow = (static_cast<size_t>(blockIdx.x) * 2 + slot) * cols;
+        for (int idx = threadIdx.x; idx < cols * D / 2; idx += kConsumerWarps * 32) {
+          const int c = (2 * idx) / D;  // column: token c / g, head c % g
           const int d = (2 * idx) % D;
           float mm = -INFINITY;
 #pragma unroll
-          for (int w = 0; w < kConsumerWarps; ++w) mm = fmaxf(mm, m_all[w * kMaxGroup + j]);
+          for (int w = 0; w < kConsumerWarps; ++w) mm = fmaxf(mm, m_all[w * kC + c]);
           float ll = 0.f, v0 = 0.f, v1 = 0.f;
 #pragma unroll
           for (int w = 0; w < kConsumerWarps; ++w) {
-            const float mw = m_all[w * kMaxGroup + j];
+            const float mw = m_all[w * kC + c];
             const float f = (mw == -INFINITY) ? 0.f : exp2f(mw - mm);
-            const float* ow = o_all + (w * kMaxGroup + j) * geo::kOStride + d;
-            ll = fmaf(f, l_all[w * kMaxGroup + j], ll);
+            const float* ow = o_all + (w * kC + c) * geo::kOStride + d;
+            ll = fmaf(f, l_all[w * kC + c], ll);
             v0 = fmaf(f, ow[0], v0);
             v1 = fmaf(f, ow[1], v1);
           }
           if (complete) {
-            const float inv = 1.f / ll;
-            *reinterpret_cast<__nv_bfloat162*>(a.out + (head0 + j) * D + d) =
+            // a query token that sees no position (len < T) gets 0
+            const float inv = ll > 0.f ? 1.f / ll : 0.f;
+            const int t = c / g;
+            *reinterpret_cast<__nv_bfloat162*>(a.out + (qrow0 + t * a.num_q_heads + (c - t * g)) * D + d) =
                 __floats2bfloat162_rn(v0 * inv, v1 * inv);
           } else {
-            *reinterpret_cast<float2*>(a.part_o + (prow + j) * D + d) = make_float2(v0, v1);
+            *reinterpret_cast<float2*>(a.part_o + (prow + c) * D + d) = make_float2(v0, v1);
             if (d == 0) {
-              a.part_m[prow + j] = mm;
-              a.part_l[prow + j] = ll;
+              a.part_m[prow + c] = mm;
+              a.part_l[prow + c] = ll;
             }
           }
         }
@@ -948,7 +1004,7 @@ __global__ void __launch_bounds__(kThreads, kStreamCtasPerSm)
   }
 }
 
-// Merge for the balanced schedule: one warp per (request, query head).  A
+// Merge for the balanced schedule: one warp per (request, query token, query head).  A
 // (b, h) covered by a single CTA was written directly; a (b, h) split across
 // CTAs c_first..c_last is merged from their partial slots (slot 0 when the
 // (b, h) is the CTA's first segment, else slot 1).  CTAs with an empty range
@@ -962,15 +1018,18 @@ __global__ void __launch_bounds__(128) paged_decode_stream_merge_kernel(const De
   constexpr int kUnroll = 8;
   pdl_trigger();
   pdl_wait();
-  const int gw = blockIdx.x * 4 + (threadIdx.x >> 5);
+  const int gw = blockIdx.x * 4 + (threadIdx.x >> 5);  // (request, token, query head)
   const int lane = threadIdx.x & 31;
   const int hkv = a.num_kv_heads;
   const int g = a.group;
-  if (gw >= batch * a.num_q_heads) return;
-  const int b = gw / a.num_q_heads;
-  const int qh = gw - b * a.num_q_heads;  // query head
-  const int h = qh / g;                   // its KV head
-  const int j = qh - h * g;               // its place in the group
+  const int per_req = a.qtok * a.num_q_heads;
+  if (gw >= batch * per_req) return;
+  const int b = gw / per_req;
+  const int t = (gw - b * per_req) / a.num_q_heads;
+  const int qh = gw - b * per_req - t * a.num_q_heads;  // query head
+  const int h = qh / g;                                 // its KV head
+  const int j = t * g + (qh - h * g);                   // its column in the (token, head) tile
+  const int cols = a.cols;
   const int* prefix = a.stream_prefix;
   const int pb0 = prefix[b], pb1 = prefix[b + 1], pall = prefix[batch];
   const int nb = pb1 - pb0;
@@ -986,11 +1045,11 @@ __global__ void __launch_bounds__(128) paged_decode_stream_merge_kernel(const De
   const int c0 = stream_cta_of(total, us, ctas);
   const int c1 = stream_cta_of(total, us + nb - 1, ctas);
   if (c0 == c1) return;  // one CTA held the whole (b, h) and wrote the output
-  // partial row of CTA c for this (b, h) and group member j, or -1 if c holds no units
+  // partial row of CTA c for this (b, h) and column j, or -1 if c holds no units
   auto row_of = [&](int c) -> long long {
     const long long cb = stream_begin(total, c, ctas);
     if (stream_begin(total, c + 1, ctas) <= cb) return -1;
-    return (static_cast<long long>(c) * 2 + (cb >= us ? 0 : 1)) * g + j;
+    return (static_cast<long long>(c) * 2 + (cb >= us ? 0 : 1)) * cols + j;
   };
   float mm = -INFINITY, den = 0.f;
   {
@@ -1051,14 +1110,15 @@ __global__ void __launch_bounds__(128) paged_decode_stream_merge_kernel(const De
     }
 #pragma unroll
     for (int q = 0; q < kUnroll; ++q) {
-      if (ok[q]) {
+      // a partial whose column saw no position has m = -inf and O = 0
+      if (ok[q] && w[q] != -INFINITY) {
         const float wq = exp2f(w[q] - mm);
 #pragma unroll
         for (int e = 0; e < kPer; ++e) acc[e] = fmaf(wq, v[q][e], acc[e]);
       }
     }
   }
-  const float inv = 1.f / den;
+  const float inv = den > 0.f ? 1.f / den : 0.f;  // a token that sees nothing gets 0
 #pragma unroll
   for (int e = 0; e < kPer; e += 2)
     *reinterpret_cast<__nv_bfloat162*>(o + e) = __floats2bfloat162_rn(acc[e] * inv, acc[e + 1] * inv);
@@ -1160,9 +1220,12 @@ static size_t align256(size_t x) { return (x + 255) & ~static_cast<size_t>(255);
 // partitions of that many tokens.
 constexpr int kForceBalanced = -1;
 static int make_plan(int batch, int hq, int hkv, int d, int bs, int max_seq_len,
-                     int partition_tokens, Plan* plan) {
+                     int partition_tokens, Plan* plan, int qtok = 1) {
   const int nblk_max = max_seq_len > 0 ? (max_seq_len + bs - 1) / bs : 1;
   const int group = hq / hkv;
+  if (qtok > 1 && partition_tokens > 0)
+    return fail(PA_ERR_UNSUPPORTED, "multi-token decode runs on the balanced schedule only");
+  if (qtok > 1) partition_tokens = kForceBalanced;
   const int sms = sm_count() > 0 ? sm_count() : 148;
   // the balanced schedule pays when there are at least a few blocks per
   // persistent CTA; tiny batches (launch-bound anyway) take the grid
@@ -1176,7 +1239,7 @@ static int make_plan(int batch, int hq, int hkv, int d, int bs, int max_seq_len,
     plan->ctas = sms * kStreamCtasPerSm;
     plan->part_blocks = 1;  // set per call from max_blocks_per_seq
     plan->max_parts = 1;
-    const size_t rows = static_cast<size_t>(plan->ctas) * 2 * group;
+    const size_t rows = static_cast<size_t>(plan->ctas) * 2 * group * qtok;
     plan->off_m = align256(rows * d * sizeof(float));
     plan->off_l = plan->off_m + align256(rows * sizeof(float));
     plan->off_prefix = plan->off_l + align256(rows * sizeof(float));
@@ -1239,16 +1302,16 @@ static int launch_main(const CUtensorMap& map, const DecodeArgs& a, int batch, c
   return PA_OK;
 }
 
-template <int D, int BS, int VAR, int G>
+template <int D, int BS, int VAR, int G, int NT = 1>
 static int launch_stream(const CUtensorMap& map, const DecodeArgs& a, int batch, int ctas,
                          cudaStream_t st) {
-  using sm = StreamSmem<D, BS, G>;
-  auto kern = paged_decode_stream_kernel<D, BS, VAR, G>;
+  using sm = StreamSmem<D, BS, G, NT>;
+  auto kern = paged_decode_stream_kernel<D, BS, VAR, G, NT>;
   const int smem = sm::dynamic_bytes(batch);
   int rc = set_smem_attr(reinterpret_cast<const void*>(kern), smem);
   if (rc != PA_OK) return rc;
   PA_CUDA_TRY(launch_pdl(kern, dim3(static_cast<unsigned>(ctas)), dim3(kThreads), smem, st, map, a, batch));
-  const int warps = batch * a.num_q_heads;
+  const int warps = batch * a.qtok * a.num_q_heads;
   PA_CUDA_TRY(launch_pdl(paged_decode_stream_merge_kernel<D>, dim3((warps + 3) / 4), dim3(128), 0, st,
                          a, batch, ctas));
   return PA_OK;
@@ -1258,7 +1321,8 @@ template <int D, int BS>
 static int dispatch(const CUtensorMap& map, const DecodeArgs& a, int batch, int variant,
                     const Plan& plan, cudaStream_t st) {
   if (plan.stream) {
-    if (variant == kMma) return launch_stream<D, BS, kMma, 0>(map, a, batch, plan.ctas, st);
+    if (variant == kMma && a.cols > 8) return launch_stream<D, BS, kMma, 0, 2>(map, a, batch, plan.ctas, st);
+    if (variant == kMma) return launch_stream<D, BS, kMma, 0, 1>(map, a, batch, plan.ctas, st);
     switch (a.group) {
       case 1: return launch_stream<D, BS, kCudaCore, 1>(map, a, batch, plan.ctas, st);
       case 2: return launch_stream<D, BS, kCudaCore, 2>(map, a, batch, plan.ctas, st);
@@ -1292,7 +1356,7 @@ static int decode_impl(pa_bf16* out, const pa_bf16* q, const pa_bf16* kv_pool,
                        const int32_t* block_tables, const int32_t* seq_lens, int batch, int hq,
                        int hkv, int d, int bs, int num_blocks, int max_blocks, int max_seq_len,
                        float scale, void* workspace, size_t ws_bytes, int variant,
-                       int partition_tokens, void* stream) {
+                       int partition_tokens, void* stream, int qtok = 1) {
   int rc = check_shape(batch, hq, hkv, d, bs, max_seq_len);
   if (rc != PA_OK) return rc;
   if (num_blocks <= 0 || max_blocks <= 0)
@@ -1308,14 +1372,20 @@ static int decode_impl(pa_bf16* out, const pa_bf16* q, const pa_bf16* kv_pool,
       (reinterpret_cast<uintptr_t>(seq_lens) & 3u))
     return fail(PA_ERR_INVALID, "pa_decode: misaligned pointer");
   const int group = hq / hkv;
-  if (variant == PA_DECODE_AUTO) variant = group >= 4 ? kMma : kCudaCore;
+  if (qtok < 1) return fail(PA_ERR_INVALID, "num_query_tokens %d below 1", qtok);
+  if (group * qtok > 2 * kMaxGroup)
+    return fail(PA_ERR_UNSUPPORTED, "group %d x query tokens %d above %d columns", group, qtok,
+                2 * kMaxGroup);
+  if (qtok > 1 && variant == kCudaCore)
+    return fail(PA_ERR_UNSUPPORTED, "multi-token decode has the tensor-core variant only");
+  if (variant == PA_DECODE_AUTO) variant = (group >= 4 || qtok > 1) ? kMma : kCudaCore;
   if (variant == kCudaCore && group != 1 && group != 2 && group != 4)
     return fail(PA_ERR_UNSUPPORTED, "pa_decode: CUDA-core variant has no group size %d", group);
   if (variant != kCudaCore && variant != kMma)
     return fail(PA_ERR_INVALID, "pa_decode: unknown variant %d", variant);
 
   Plan plan;
-  rc = make_plan(batch, hq, hkv, d, bs, max_seq_len, partition_tokens, &plan);
+  rc = make_plan(batch, hq, hkv, d, bs, max_seq_len, partition_tokens, &plan, qtok);
   if (rc != PA_OK) return rc;
   if (plan.bytes > 0) {
     if (workspace == nullptr || ws_bytes < plan.bytes)
@@ -1357,6 +1427,8 @@ static int decode_impl(pa_bf16* out, const pa_bf16* q, const pa_bf16* kv_pool,
   a.max_parts = plan.max_parts;
   a.scale_log2 = scale * 1.4426950408889634f;
   a.stream_prefix = plan.stream ? reinterpret_cast<int*>(ws + plan.off_prefix) : nullptr;
+  a.qtok = qtok;
+  a.cols = group * qtok;
 
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   if (d == 64 && bs == 16) return dispatch<64, 16>(map, a, batch, variant, plan, st);
@@ -1386,6 +1458,35 @@ int pa_decode_workspace_size_ex(int batch, int num_q_heads, int num_kv_heads, in
   if (num_partitions_out) *num_partitions_out = plan.stream ? plan.ctas : plan.max_parts;
   if (balanced_out) *balanced_out = plan.stream ? 1 : 0;
   return PA_OK;
+}
+
+int pa_decode_multi_workspace_size(int batch, int num_query_tokens, int num_q_heads,
+                                   int num_kv_heads, int head_dim, int block_size,
+                                   int max_seq_len, size_t* bytes_out) {
+  using namespace pa;
+  if (bytes_out == nullptr) return fail(PA_ERR_INVALID, "pa_decode_multi_workspace_size: NULL bytes_out");
+  int rc = check_shape(batch, num_q_heads, num_kv_heads, head_dim, block_size, max_seq_len);
+  if (rc != PA_OK) return rc;
+  if (num_query_tokens < 1) return fail(PA_ERR_INVALID, "num_query_tokens %d below 1", num_query_tokens);
+  if (num_q_heads / num_kv_heads * num_query_tokens > 2 * kMaxGroup)
+    return fail(PA_ERR_UNSUPPORTED, "group x query tokens above %d columns", 2 * kMaxGroup);
+  Plan plan;
+  rc = make_plan(batch, num_q_heads, num_kv_heads, head_dim, block_size, max_seq_len, kForceBalanced,
+                 &plan, num_query_tokens);
+  if (rc != PA_OK) return rc;
+  *bytes_out = plan.bytes;
+  return PA_OK;
+}
+
+int pa_decode_multi(pa_bf16* out, const pa_bf16* q, const pa_bf16* kv_pool,
+                    const int32_t* block_tables, const int32_t* seq_lens, int batch,
+                    int num_query_tokens, int num_q_heads, int num_kv_heads, int head_dim,
+                    int block_size, int num_blocks, int max_blocks_per_seq, int max_seq_len,
+                    float scale, void* workspace, size_t workspace_bytes, void* stream) {
+  return pa::decode_impl(out, q, kv_pool, block_tables, seq_lens, batch, num_q_heads, num_kv_heads,
+                         head_dim, block_size, num_blocks, max_blocks_per_seq, max_seq_len, scale,
+                         workspace, workspace_bytes, PA_DECODE_MMA, pa::kForceBalanced, stream,
+                         num_query_tokens);
 }
 
 int pa_decode_workspace_size(int batch, int num_q_heads, int num_kv_heads, int head_dim,
