@@ -605,6 +605,48 @@ def study_page_table(iters=30):
     assert pk.pa_device_error() == 0
 
 
+def study_multi_token(iters=30):
+    """pa_decode_multi at the llama8b shape for T = 1, 2, 4 causal query
+    tokens per request (speculative verification): KV bytes stay the same,
+    the tensor-core tile widens from 4 to 16 (token, head) columns."""
+    import torch
+
+    import paged_kv_cache_354_b200 as pk
+
+    dev = torch.device("cuda", torch.cuda.current_device())
+    p, cache, ids, gen = build_cache("llama8b", 8, 0, dev)
+    tables, lens = cache.alloc.block_tables(ids, cache.max_blocks)
+    d_t, d_l = torch.as_tensor(tables, device=dev), torch.as_tensor(lens, device=dev)
+    nbytes = decode_bytes(lens, cache.hq, cache.hkv, cache.d, cache.bs)[0]
+    for T in (1, 2, 4):
+        q = torch.randn((len(ids), T, cache.hq, cache.d), generator=gen, device=dev).bfloat16()
+        out = torch.empty_like(q)
+        ws = torch.empty(max(256, pk.pa_decode_multi_workspace_size(len(ids), T, cache.hq, cache.hkv, cache.d,
+                                                                     cache.bs, cache.max_seq_len)),
+                         dtype=torch.uint8, device=dev)
+
+        def call():
+            pk.pa_decode_multi(out, q, cache.pool, d_t, d_l, cache.max_seq_len, 1.0 / math.sqrt(cache.d), ws)
+
+        for _ in range(3):
+            call()
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        for _ in range(iters):
+            call()
+        e1.record()
+        torch.cuda.synchronize()
+        us = e0.elapsed_time(e1) / iters * 1e3
+        extra_qo = 2 * len(ids) * (T - 1) * cache.hq * cache.d * 2
+        print(json.dumps({"study": "multi_token", "workload": "llama8b", "query_tokens": T,
+                          "columns_per_kv_head": T * cache.hq // cache.hkv, "us": round(us, 2),
+                          "gbs": round((nbytes + extra_qo) / us / 1e3, 1),
+                          "frac_of_hbm_peak": round((nbytes + extra_qo) / us / 1e3 / load_peaks()["hbm_gbs"], 4),
+                          "tokens_per_s": round(len(ids) * T / us * 1e6, 1)}), flush=True)
+    assert pk.pa_device_error() == 0
+
+
 def main():
     ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
     ap.add_argument("--gpus", type=int, default=1)
@@ -614,7 +656,7 @@ def main():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--variant", default="auto", choices=["auto", "mma", "cuda_core"],
                     help="decode consumer: auto (tensor cores for GQA groups >= 4), or forced")
-    ap.add_argument("--study", choices=["memory-waste", "page-table"],
+    ap.add_argument("--study", choices=["memory-waste", "page-table", "multi-token"],
                     help="print the study's JSON lines instead of the benchmark line")
     ap.add_argument("--partition-tokens", type=int, default=0,
                     help="0 = library's choice; -1 = balanced schedule; N > 0 = per-partition grid of "
@@ -628,6 +670,8 @@ def main():
         study_memory_waste()
     elif args.study == "page-table":
         study_page_table()
+    elif args.study == "multi-token":
+        study_multi_token()
     elif args.impl == "reference":
         run_reference(args)
     else:
