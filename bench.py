@@ -264,16 +264,11 @@ def run_gpu(args):
     if world > 1:
         dist.barrier()
     start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    from paged_kv_cache_354_b200 import pa_copy_blocks, pa_reshape_and_cache
-
     with ClockSampler(device.index) as clocks:
         start.record(stream)
         for i in range(W, W + K):
             j = i % INPUT_SETS
-            if d_pairs[i].shape[0]:
-                pa_copy_blocks(cache.pool, d_pairs[i])
-            pa_reshape_and_cache(ks[j], vs[j], cache.pool, d_slots[i])
-            cache.decode(qs[j], out, d_tables[i], d_lens[i])
+            cache.run(qs[j], ks[j], vs[j], out, d_slots[i], d_tables[i], d_lens[i], d_pairs[i])
         end.record(stream)
         torch.cuda.synchronize()
         # the dominant kernel alone: K back-to-back decode launches (main + merge)

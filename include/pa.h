@@ -235,6 +235,31 @@ int pa_decode_noalloc(pa_bf16* out, const pa_bf16* q, const pa_bf16* kv_pool,
                       void* stream);
 
 /* --------------------------------------------------------------------------
+ * pa_decode_append -- pa_reshape_and_cache of each request's newest token,
+ * then pa_decode, in one pass.
+ *
+ * The same results as pa_reshape_and_cache(new_k, new_v, kv_pool,
+ * slot_mapping, batch, ...) followed by pa_decode(...) on the same stream,
+ * for the decode step where every request has just appended one token
+ * ("Paged attention in LLMs", section "The cache being stored"): request
+ * b's new token is its position seq_lens[b] - 1 and slot_mapping[b] must be
+ * that position's slot (block_tables[b][(L-1)/bs] * bs + (L-1) % bs, as
+ * pa_alloc_append returns it); a negative slot writes nothing.  On the
+ * balanced schedule the decode kernel puts the new row straight into the
+ * staged tile and the merge kernel stores it in the pool afterwards (no
+ * separate cache-write launch); otherwise the two kernels run in turn.
+ * new_k, new_v : device bf16 [batch][num_kv_heads][head_dim]
+ * slot_mapping : device int64 [batch]
+ * Other arguments, workspace and limits as pa_decode.
+ * ------------------------------------------------------------------------ */
+int pa_decode_append(pa_bf16* out, const pa_bf16* q, pa_bf16* kv_pool, const pa_bf16* new_k,
+                     const pa_bf16* new_v, const int64_t* slot_mapping, const int32_t* block_tables,
+                     const int32_t* seq_lens, int batch, int num_q_heads, int num_kv_heads,
+                     int head_dim, int block_size, int num_blocks, int max_blocks_per_seq,
+                     int max_seq_len, float scale, void* workspace, size_t workspace_bytes,
+                     void* stream);
+
+/* --------------------------------------------------------------------------
  * pa_decode_multi -- several query tokens per request, causal.
  *
  * The single-token operation above, for the T newest tokens of each request

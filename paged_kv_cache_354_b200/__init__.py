@@ -61,6 +61,8 @@ _SIGNATURES = {
     "pa_decode_ex": (_I, [_P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _I, _I, _c.c_float, _P, _SZ,
                           _I, _I, _P]),
     "pa_decode_noalloc": (_I, [_P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _I, _I, _c.c_float, _P]),
+    "pa_decode_append": (_I, [_P, _P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _I, _I, _c.c_float, _P,
+                              _SZ, _P]),
     "pa_decode_multi_workspace_size": (_I, [_I, _I, _I, _I, _I, _I, _I, _P]),
     "pa_decode_multi": (_I, [_P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _I, _I, _I, _c.c_float, _P, _SZ,
                              _P]),
@@ -269,6 +271,32 @@ def pa_decode_noalloc(out, q, kv_pool, block_tables, seq_lens, max_seq_len, scal
     _check(lib.pa_decode_noalloc(_ptr(out), _ptr(q), _ptr(kv_pool), _ptr(block_tables), _ptr(seq_lens), b,
                                  hq, hkv, d, bs, nb, block_tables.shape[1], int(max_seq_len), float(scale),
                                  _stream(stream)), "pa_decode_noalloc")
+
+
+def pa_decode_append(out, q, kv_pool, key, value, slot_mapping, block_tables, seq_lens, max_seq_len, scale,
+                     workspace=None, stream=None):
+    """pa_reshape_and_cache of each request's newest token (key/value
+    [B, Hkv, D], slot_mapping [B]) and pa_decode, in one pass."""
+    import torch
+
+    for t, dt, n in ((out, torch.bfloat16, "out"), (q, torch.bfloat16, "q"), (kv_pool, torch.bfloat16, "kv_pool"),
+                     (key, torch.bfloat16, "key"), (value, torch.bfloat16, "value"),
+                     (slot_mapping, torch.int64, "slot_mapping"), (block_tables, torch.int32, "block_tables"),
+                     (seq_lens, torch.int32, "seq_lens")):
+        _require(t, dt, n)
+    nb, two, hkv, bs, d = kv_pool.shape
+    b, hq, dq = q.shape
+    if (out.shape != q.shape or dq != d or key.shape != (b, hkv, d) or value.shape != (b, hkv, d)
+            or slot_mapping.shape != (b,) or block_tables.shape[0] != b or seq_lens.shape != (b,)):
+        raise ValueError("pa_decode_append: shape mismatch")
+    ws_ptr, ws_bytes = None, 0
+    if workspace is not None:
+        _require(workspace, torch.uint8, "workspace")
+        ws_ptr, ws_bytes = _ptr(workspace), workspace.numel()
+    _check(lib.pa_decode_append(_ptr(out), _ptr(q), _ptr(kv_pool), _ptr(key), _ptr(value), _ptr(slot_mapping),
+                                _ptr(block_tables), _ptr(seq_lens), b, hq, hkv, d, bs, nb, block_tables.shape[1],
+                                int(max_seq_len), float(scale), ws_ptr, ws_bytes, _stream(stream)),
+           "pa_decode_append")
 
 
 def pa_selftest_wait_timeout(limit_ns, stream=None):

@@ -91,6 +91,13 @@ struct DecodeArgs {
   int* stream_prefix;  // balanced schedule: per-request block-count prefix sums [B+1]
   int qtok;            // query tokens per request (1 = single-token decode)
   int cols;            // group * qtok: (token, head) columns per KV head
+  // fused cache write (pa_decode_append): request b's newest token, at
+  // position seq_lens[b] - 1, has keys/values new_k/new_v [B][Hkv][D] and
+  // slot new_slots[b] (< 0: nothing to write); null when not fused
+  const uint4* new_k;
+  const uint4* new_v;
+  const int64_t* new_slots;
+  uint4* pool_w;       // the pool, written by the merge kernel
 };
 
 // Tokens of request b the kernels attend over, after the device-side checks
@@ -928,6 +935,19 @@ __global__ void __launch_bounds__(kThreads, kStreamCtasPerSm)
       const __nv_bfloat16* qbase = a.q + qrow0 * D;
       if constexpr (VAR == kMma) mc.init(qbase, cols, g, a.qtok, q_tok_stride, len, lane);
       else cc.init(qbase, lane);
+      // fused cache write: the warp that takes this (b, h)'s last block
+      // fetches the new K/V row now and patches it into the staged tile
+      const int last_ii = i + cnt - 1;
+      bool patch = false;
+      uint4 new_row = make_uint4(0u, 0u, 0u, 0u);
+      if (a.new_k != nullptr && k + cnt == nb && last_ii % kConsumerWarps == warp) {
+        patch = __ldg(a.new_slots + b) >= 0;
+        if (patch && lane < 2 * (D / 8)) {
+          const uint4* src = (lane < D / 8 ? a.new_k : a.new_v) +
+                             (static_cast<size_t>(b) * hkv + h) * (D / 8) + lane % (D / 8);
+          new_row = __ldg(src);
+        }
+      }
       // this warp's blocks of the segment: running indices i..i+cnt-1 that are
       // congruent to the warp number
       for (int ii = i + ((warp - i % kConsumerWarps + kConsumerWarps) % kConsumerWarps);
@@ -944,6 +964,21 @@ __global__ void __launch_bounds__(kThreads, kStreamCtasPerSm)
         const uint32_t sb = sbase + s * geo::kStageBytes;
         const int blk = k + (ii - i);
         const int valid = (blk == nb - 1) ? last_valid : BS;
+        if (patch && ii == last_ii) {
+          // row of position len - 1: K row in the K half, V row in the V half
+          if (lane < 2 * (D / 8)) {
+            const int kv = lane / (D / 8);
+            const int chunk = lane % (D / 8);
+            const int r = valid - 1;
+            const uint32_t addr = sb + (chunk >> 3) * geo::kRegionBytes + (kv * BS + r) * 128 +
+                                  (((chunk & 7) ^ (r & 7)) << 4);
+            asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(new_row.x),
+                         "r"(new_row.y), "r"(new_row.z), "r"(new_row.w)
+                         : "memory");
+          }
+          fence_proxy_async_smem();  // the stage goes back to TMA later
+          __syncwarp();
+        }
         consume_block<D, BS, VAR, G, NT>(mc, cc, sb, pbuf, valid, blk * BS, a.scale_log2, lane);
         __syncwarp();
         if (lane == 0) mbar_arrive(bar_empty + 8 * s);
@@ -1011,7 +1046,7 @@ __global__ void __launch_bounds__(kThreads, kStreamCtasPerSm)
 // (more CTAs than units) wrote nothing and are skipped.  Requests of length
 // 0 get zeros here.  Three dependent memory rounds per warp: the prefix
 // sums, every CTA's (m, l) (one per lane), then all partial O rows at once.
-template <int D>
+template <int D, int BS>
 __global__ void __launch_bounds__(128) paged_decode_stream_merge_kernel(const DecodeArgs a,
                                                                         int batch, int ctas) {
   constexpr int kPer = D / 32;
@@ -1030,6 +1065,22 @@ __global__ void __launch_bounds__(128) paged_decode_stream_merge_kernel(const De
   const int h = qh / g;                                 // its KV head
   const int j = t * g + (qh - h * g);                   // its column in the (token, head) tile
   const int cols = a.cols;
+  if (a.new_k != nullptr && t == 0 && qh == h * g && lane < 2 * (D / 8)) {
+    // fused cache write: the decode kernel has finished reading the pool,
+    // so request b's new K/V row for KV head h lands in its slot now
+    const long long slot = __ldg(a.new_slots + b);
+    const long long nslots = static_cast<long long>(a.num_blocks) * BS;
+    if (slot >= nslots) {
+      if (lane == 0) flag_error(a.err, PA_DEVERR_SLOT);
+    } else if (slot >= 0) {
+      const int kv = lane / (D / 8);
+      const int chunk = lane % (D / 8);
+      const long long blk = slot / BS;
+      const long long off = slot - blk * BS;
+      const uint4* src = (kv ? a.new_v : a.new_k) + (static_cast<size_t>(b) * hkv + h) * (D / 8) + chunk;
+      a.pool_w[(((blk * 2 + kv) * hkv + h) * BS + off) * (D / 8) + chunk] = __ldg(src);
+    }
+  }
   const int* prefix = a.stream_prefix;
   const int pb0 = prefix[b], pb1 = prefix[b + 1], pall = prefix[batch];
   const int nb = pb1 - pb0;
@@ -1312,7 +1363,7 @@ static int launch_stream(const CUtensorMap& map, const DecodeArgs& a, int batch,
   if (rc != PA_OK) return rc;
   PA_CUDA_TRY(launch_pdl(kern, dim3(static_cast<unsigned>(ctas)), dim3(kThreads), smem, st, map, a, batch));
   const int warps = batch * a.qtok * a.num_q_heads;
-  PA_CUDA_TRY(launch_pdl(paged_decode_stream_merge_kernel<D>, dim3((warps + 3) / 4), dim3(128), 0, st,
+  PA_CUDA_TRY(launch_pdl(paged_decode_stream_merge_kernel<D, BS>, dim3((warps + 3) / 4), dim3(128), 0, st,
                          a, batch, ctas));
   return PA_OK;
 }
@@ -1356,7 +1407,9 @@ static int decode_impl(pa_bf16* out, const pa_bf16* q, const pa_bf16* kv_pool,
                        const int32_t* block_tables, const int32_t* seq_lens, int batch, int hq,
                        int hkv, int d, int bs, int num_blocks, int max_blocks, int max_seq_len,
                        float scale, void* workspace, size_t ws_bytes, int variant,
-                       int partition_tokens, void* stream, int qtok = 1) {
+                       int partition_tokens, void* stream, int qtok = 1,
+                       const pa_bf16* new_k = nullptr, const pa_bf16* new_v = nullptr,
+                       const int64_t* new_slots = nullptr) {
   int rc = check_shape(batch, hq, hkv, d, bs, max_seq_len);
   if (rc != PA_OK) return rc;
   if (num_blocks <= 0 || max_blocks <= 0)
@@ -1371,6 +1424,13 @@ static int decode_impl(pa_bf16* out, const pa_bf16* q, const pa_bf16* kv_pool,
   if (!a16(out) || !a16(q) || !a16(kv_pool) || (reinterpret_cast<uintptr_t>(block_tables) & 3u) ||
       (reinterpret_cast<uintptr_t>(seq_lens) & 3u))
     return fail(PA_ERR_INVALID, "pa_decode: misaligned pointer");
+  const bool fused = new_k != nullptr;
+  if (fused) {
+    if (!new_v || !new_slots) return fail(PA_ERR_INVALID, "pa_decode_append: NULL new_v or slot_mapping");
+    if (!a16(new_k) || !a16(new_v) || (reinterpret_cast<uintptr_t>(new_slots) & 7u))
+      return fail(PA_ERR_INVALID, "pa_decode_append: misaligned pointer");
+    if (qtok != 1) return fail(PA_ERR_UNSUPPORTED, "pa_decode_append: one new token per request");
+  }
   const int group = hq / hkv;
   if (qtok < 1) return fail(PA_ERR_INVALID, "num_query_tokens %d below 1", qtok);
   if (group * qtok > 2 * kMaxGroup)
@@ -1429,8 +1489,23 @@ static int decode_impl(pa_bf16* out, const pa_bf16* q, const pa_bf16* kv_pool,
   a.stream_prefix = plan.stream ? reinterpret_cast<int*>(ws + plan.off_prefix) : nullptr;
   a.qtok = qtok;
   a.cols = group * qtok;
-
+  a.new_k = nullptr;
+  a.new_v = nullptr;
+  a.new_slots = nullptr;
+  a.pool_w = reinterpret_cast<uint4*>(const_cast<pa_bf16*>(kv_pool));
   cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (fused) {
+    if (plan.stream) {  // the decode kernel patches, the merge kernel writes
+      a.new_k = reinterpret_cast<const uint4*>(new_k);
+      a.new_v = reinterpret_cast<const uint4*>(new_v);
+      a.new_slots = new_slots;
+    } else {  // per-partition grid: the cache write runs first, on its own
+      rc = pa_reshape_and_cache(new_k, new_v, const_cast<pa_bf16*>(kv_pool), new_slots, batch,
+                                num_blocks, hkv, bs, d, stream);
+      if (rc != PA_OK) return rc;
+    }
+  }
+
   if (d == 64 && bs == 16) return dispatch<64, 16>(map, a, batch, variant, plan, st);
   if (d == 64 && bs == 32) return dispatch<64, 32>(map, a, batch, variant, plan, st);
   if (d == 128 && bs == 16) return dispatch<128, 16>(map, a, batch, variant, plan, st);
@@ -1487,6 +1562,20 @@ int pa_decode_multi(pa_bf16* out, const pa_bf16* q, const pa_bf16* kv_pool,
                          head_dim, block_size, num_blocks, max_blocks_per_seq, max_seq_len, scale,
                          workspace, workspace_bytes, PA_DECODE_MMA, pa::kForceBalanced, stream,
                          num_query_tokens);
+}
+
+int pa_decode_append(pa_bf16* out, const pa_bf16* q, pa_bf16* kv_pool, const pa_bf16* new_k,
+                     const pa_bf16* new_v, const int64_t* slot_mapping, const int32_t* block_tables,
+                     const int32_t* seq_lens, int batch, int num_q_heads, int num_kv_heads,
+                     int head_dim, int block_size, int num_blocks, int max_blocks_per_seq,
+                     int max_seq_len, float scale, void* workspace, size_t workspace_bytes,
+                     void* stream) {
+  if (batch > 0 && (new_k == nullptr || new_v == nullptr || slot_mapping == nullptr))
+    return pa::fail(PA_ERR_INVALID, "pa_decode_append: NULL new_k, new_v or slot_mapping");
+  return pa::decode_impl(out, q, kv_pool, block_tables, seq_lens, batch, num_q_heads, num_kv_heads,
+                         head_dim, block_size, num_blocks, max_blocks_per_seq, max_seq_len, scale,
+                         workspace, workspace_bytes, PA_DECODE_AUTO, 0, stream, 1, new_k, new_v,
+                         slot_mapping);
 }
 
 int pa_decode_workspace_size(int batch, int num_q_heads, int num_kv_heads, int head_dim,

@@ -21,7 +21,7 @@ import ctypes
 import numpy as np
 import torch
 
-from . import (PA_DECODE_AUTO, PaAlloc, _check, lib, pa_copy_blocks, pa_decode,
+from . import (PA_DECODE_AUTO, PaAlloc, _check, lib, pa_copy_blocks, pa_decode, pa_decode_append,
                pa_decode_workspace_size, pa_reshape_and_cache)
 
 
@@ -130,8 +130,7 @@ class PagedDecodeCache:
         return g
 
     def _device_step(self, q, k_new, v_new, out):
-        pa_reshape_and_cache(k_new, v_new, self.pool, self.s_slots)
-        self.decode(q, out, self.s_tables, self.s_lens)
+        self.append_decode(q, k_new, v_new, out, self.s_slots, self.s_tables, self.s_lens)
 
     def replay(self, npairs):
         """Device part of a staged step: copy-on-write copies (if any), then the graph."""
@@ -141,11 +140,22 @@ class PagedDecodeCache:
 
     # -------------------------------------------------------------- device
     def run(self, q, k_new, v_new, out, slots, tables, lens, pairs=None, max_seq_len=None):
-        """Device part of a step on already-resident inputs (async)."""
+        """Device part of a step on already-resident inputs (async): the
+        copy-on-write copies, then the new tokens' cache write fused with the
+        decode (pa_decode_append; the library's default path).  With an
+        explicit partition size or variant the two calls run separately."""
         if pairs is not None and pairs.shape[0] > 0:
             pa_copy_blocks(self.pool, pairs)
-        pa_reshape_and_cache(k_new, v_new, self.pool, slots)
-        self.decode(q, out, tables, lens, max_seq_len)
+        self.append_decode(q, k_new, v_new, out, slots, tables, lens, max_seq_len)
+
+    def append_decode(self, q, k_new, v_new, out, slots, tables, lens, max_seq_len=None):
+        if self.partition_tokens == 0 and self.variant == PA_DECODE_AUTO:
+            pa_decode_append(out, q, self.pool, k_new, v_new, slots, tables, lens,
+                             max_seq_len or self.max_seq_len, 1.0 / float(np.sqrt(self.d)),
+                             workspace=self.workspace)
+        else:
+            pa_reshape_and_cache(k_new, v_new, self.pool, slots)
+            self.decode(q, out, tables, lens, max_seq_len)
 
     def decode(self, q, out, tables, lens, max_seq_len=None):
         pa_decode(out, q, self.pool, tables, lens, max_seq_len or self.max_seq_len,
@@ -154,4 +164,6 @@ class PagedDecodeCache:
 
     def launches_per_step(self, npairs):
         """Kernels this library launches for one step."""
-        return (1 if npairs else 0) + 1 + 1 + (1 if self.num_partitions > 1 else 0)
+        fused = self.partition_tokens == 0 and self.variant == PA_DECODE_AUTO and self.schedule == "balanced"
+        cache_write = 0 if fused else 1
+        return (1 if npairs else 0) + cache_write + 1 + (1 if self.num_partitions > 1 else 0)
