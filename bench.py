@@ -642,6 +642,28 @@ def study_multi_token(iters=30):
     assert pk.pa_device_error() == 0
 
 
+def study_read_bandwidth(iters=20):
+    """What a plain contiguous read stream reaches on this GPU: torch's own
+    bf16 sum (fp32 accumulate) over 2 GiB, for context beside the copy-based
+    peak in MEASURED_PEAKS.json (which counts a read and a write per byte)."""
+    import torch
+
+    x = torch.empty(1024 ** 3, dtype=torch.bfloat16, device="cuda").normal_()
+    for _ in range(3):
+        torch.sum(x, dtype=torch.float32)
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for _ in range(iters):
+        torch.sum(x, dtype=torch.float32)
+    e1.record()
+    torch.cuda.synchronize()
+    ms = e0.elapsed_time(e1) / iters
+    print(json.dumps({"study": "read_bandwidth", "probe": "torch.sum bf16 -> fp32 over 2 GiB",
+                      "gbs": round(x.numel() * 2 / ms / 1e6, 1), "ms": round(ms, 4),
+                      "copy_peak_gbs": load_peaks()["hbm_gbs"]}), flush=True)
+
+
 def main():
     ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
     ap.add_argument("--gpus", type=int, default=1)
@@ -651,7 +673,7 @@ def main():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--variant", default="auto", choices=["auto", "mma", "cuda_core"],
                     help="decode consumer: auto (tensor cores for GQA groups >= 4), or forced")
-    ap.add_argument("--study", choices=["memory-waste", "page-table", "multi-token"],
+    ap.add_argument("--study", choices=["memory-waste", "page-table", "multi-token", "read-bandwidth"],
                     help="print the study's JSON lines instead of the benchmark line")
     ap.add_argument("--partition-tokens", type=int, default=0,
                     help="0 = library's choice; -1 = balanced schedule; N > 0 = per-partition grid of "
@@ -667,6 +689,8 @@ def main():
         study_page_table()
     elif args.study == "multi-token":
         study_multi_token()
+    elif args.study == "read-bandwidth":
+        study_read_bandwidth()
     elif args.impl == "reference":
         run_reference(args)
     else:

@@ -259,7 +259,7 @@ struct MmaConsumer {
 
   // Write this warp's unnormalised O, running max and sum to the epilogue
   // scratch: o_s[column][dim] (row stride kOStride), m_s[column], l_s[column].
-  __device__ __forceinline__ void store(float* o_s, float* m_s, float* l_s, int lane) {
+  __device__ __forceinline__ void store(float* o_s, float* m_s, float* l_s, int rows, int lane) {
     const int c = 2 * (lane & 3);
 #pragma unroll
     for (int nt = 0; nt < NT; ++nt) {
@@ -271,6 +271,7 @@ struct MmaConsumer {
         l[nt][e] = le;
       }
       const int c0 = nt * 8 + c;
+      if (c0 >= rows) continue;  // columns past the call's (even) column count
 #pragma unroll
       for (int dt = 0; dt < kDT; ++dt) {
         const int d = 16 * dt + (lane >> 2);
@@ -610,7 +611,7 @@ __global__ void __launch_bounds__(kThreads, (VAR == kMma || G <= 2) ? 3 : 2)
     float* o_s = reinterpret_cast<float*>(smem) + warp * kMaxGroup * geo::kOStride;
     float* m_s = reinterpret_cast<float*>(smem + geo::kEpiO) + warp * kMaxGroup;
     float* l_s = m_s + kConsumerWarps * kMaxGroup;
-    if constexpr (VAR == kMma) mc.store(o_s, m_s, l_s, lane);
+    if constexpr (VAR == kMma) mc.store(o_s, m_s, l_s, kMaxGroup, lane);
     else cc.store(o_s, m_s, l_s, lane);
   }
   __syncthreads();  // (B) epilogue scratch written
@@ -716,9 +717,20 @@ struct StreamSmem {
   static constexpr int kPbuf = kScan + (kThreads + 4) * 4;       // CUDA-core p tiles
   static constexpr int kPbufBytes = kConsumerWarps * BS * (G > 0 ? G : 1) * 4;
   static constexpr int kEpi = (kPbuf + kPbufBytes + 15) & ~15;   // per-warp O, m, l
-  static constexpr int kEpiO = kConsumerWarps * kCols * geo::kOStride * 4;
-  static constexpr int kPrefix = kEpi + kEpiO + 2 * kConsumerWarps * kCols * 4;  // int32 [batch+1]
-  static constexpr int dynamic_bytes(int batch) { return kPrefix + 4 * (batch + 1) + 1024; }
+  // the epilogue holds only the columns a call uses (group * query tokens,
+  // rounded up to a pair), so narrow groups leave room for a deeper ring
+  static __host__ __device__ constexpr int epi_rows(int cols) {
+    return cols + (cols & 1) < kCols ? cols + (cols & 1) : kCols;
+  }
+  static __host__ __device__ constexpr int epi_o_bytes(int cols) {
+    return kConsumerWarps * epi_rows(cols) * geo::kOStride * 4;
+  }
+  static __host__ __device__ constexpr int prefix_offset(int cols) {
+    return kEpi + epi_o_bytes(cols) + 2 * kConsumerWarps * epi_rows(cols) * 4;  // int32 [batch+1]
+  }
+  static constexpr int dynamic_bytes(int batch, int cols) {
+    return prefix_offset(cols) + 4 * (batch + 1) + 1024;
+  }
 };
 
 // First unit of the CTA range that contains unit u: the largest c with
@@ -835,7 +847,7 @@ __global__ void __launch_bounds__(kThreads, kStreamCtasPerSm)
   const uint32_t bar_empty = bar_full + 8 * sm::kStages;
   int* last_round = reinterpret_cast<int*>(smem + sm::kMisc);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + sm::kMisc + 4 * sm::kStages);
-  int* prefix = reinterpret_cast<int*>(smem + sm::kPrefix);
+  int* prefix = reinterpret_cast<int*>(smem + sm::prefix_offset(a.cols));
 
   if (threadIdx.x == 0) {  // shared memory only: may overlap the previous grid
     for (int s = 0; s < sm::kStages; ++s) {
@@ -913,9 +925,9 @@ __global__ void __launch_bounds__(kThreads, kStreamCtasPerSm)
   } else {
     // ----------------------------------------------------------- consumers
     float* pbuf = reinterpret_cast<float*>(smem + sm::kPbuf) + warp * BS * (G > 0 ? G : 1);
-    constexpr int kC = sm::kCols;
+    const int kC = sm::epi_rows(a.cols);  // epilogue rows per warp
     float* o_all = reinterpret_cast<float*>(smem + sm::kEpi);
-    float* m_all = reinterpret_cast<float*>(smem + sm::kEpi + sm::kEpiO);
+    float* m_all = reinterpret_cast<float*>(smem + sm::kEpi + sm::epi_o_bytes(a.cols));
     float* l_all = m_all + kConsumerWarps * kC;
     const int cols = a.cols;
     const size_t q_tok_stride = static_cast<size_t>(a.num_q_heads) * D;
@@ -986,7 +998,7 @@ __global__ void __launch_bounds__(kThreads, kStreamCtasPerSm)
       // ---- segment epilogue: merge the four warps' states
       {
         float* o_s = o_all + warp * kC * geo::kOStride;
-        if constexpr (VAR == kMma) mc.store(o_s, m_all + warp * kC, l_all + warp * kC, lane);
+        if constexpr (VAR == kMma) mc.store(o_s, m_all + warp * kC, l_all + warp * kC, kC, lane);
         else cc.store(o_s, m_all + warp * kC, l_all + warp * kC, lane);
       }
       consumer_bar();
@@ -1358,7 +1370,7 @@ static int launch_stream(const CUtensorMap& map, const DecodeArgs& a, int batch,
                          cudaStream_t st) {
   using sm = StreamSmem<D, BS, G, NT>;
   auto kern = paged_decode_stream_kernel<D, BS, VAR, G, NT>;
-  const int smem = sm::dynamic_bytes(batch);
+  const int smem = sm::dynamic_bytes(batch, a.cols);
   int rc = set_smem_attr(reinterpret_cast<const void*>(kern), smem);
   if (rc != PA_OK) return rc;
   PA_CUDA_TRY(launch_pdl(kern, dim3(static_cast<unsigned>(ctas)), dim3(kThreads), smem, st, map, a, batch));

@@ -105,6 +105,13 @@ int set_smem_attr(const void* kernel, int bytes) {
   return PA_OK;
 }
 
+// L2 fetch granularity of the TMA loads (build-time tuning; the decode
+// boxes read 128-byte halves of 256-byte rows, so 256-byte promotion brings
+// the other half into L2 with the first).
+#ifndef PA_TMA_L2_PROMOTION
+#define PA_TMA_L2_PROMOTION CU_TENSOR_MAP_L2_PROMOTION_L2_256B
+#endif
+
 int encode_tensor_map(void* desc, int rank, void* base, const uint64_t* dims,
                       const uint64_t* strides_bytes, const uint32_t* box, int swizzle_128b) {
   {
@@ -132,7 +139,7 @@ int encode_tensor_map(void* desc, int rank, void* base, const uint64_t* dims,
                         static_cast<cuuint32_t>(rank), base, d, s, b, es,
                         CU_TENSOR_MAP_INTERLEAVE_NONE,
                         swizzle_128b ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_NONE,
-                        CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+                        PA_TMA_L2_PROMOTION, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   if (r != CUDA_SUCCESS) return fail(PA_ERR_CUDA, "cuTensorMapEncodeTiled failed (CUresult %d)", (int)r);
   return PA_OK;
 }
