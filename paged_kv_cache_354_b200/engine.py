@@ -32,7 +32,7 @@ def _align(n, a=256):
 class PagedDecodeCache:
     def __init__(self, num_blocks, num_q_heads, num_kv_heads, head_dim, block_size, max_batch,
                  max_seq_len, initial_order=None, device="cuda", partition_tokens=0,
-                 variant=PA_DECODE_AUTO):
+                 variant=PA_DECODE_AUTO, staging_sets=1):
         self.num_blocks = int(num_blocks)
         self.hq, self.hkv, self.d, self.bs = num_q_heads, num_kv_heads, head_dim, block_size
         self.max_batch = int(max_batch)
@@ -48,36 +48,46 @@ class PagedDecodeCache:
             self.max_batch, num_q_heads, num_kv_heads, head_dim, block_size, self.max_seq_len,
             partition_tokens, with_schedule=True)
         self.workspace = torch.empty(max(nbytes, 256), dtype=torch.uint8, device=self.device)
-        # one pinned buffer (and its device twin) for a step's metadata:
-        # slots int64[B] | lens int32[B] | pairs int32[B,2] | tables int32[B,MB]
+        # A step's staging buffer: metadata written by the allocator and the
+        # step's inputs, in one pinned block that reaches the device in one
+        # copy.  Layout: slots int64[B] | lens int32[B] | pairs int32[B,2] |
+        # tables int32[B,MB] | q bf16[B,Hq,D] | k bf16[B,Hkv,D] | v bf16[B,Hkv,D].
+        # ``staging_sets`` pinned buffers rotate so a caller can fill the
+        # next step's inputs while the device works on the current one.
         b, mb = self.max_batch, self.max_blocks
         self._layout = {}
         off = 0
-        for name, dtype, count in (("slots", torch.int64, b), ("lens", torch.int32, b),
-                                   ("pairs", torch.int32, 2 * b), ("tables", torch.int32, b * mb)):
-            self._layout[name] = (off, dtype, count)
-            off += _align(count * torch.empty((), dtype=dtype).element_size())
-        self.meta_bytes = off
-        self.h_meta = torch.zeros(off, dtype=torch.uint8).pin_memory()
-        self.d_meta = torch.zeros(off, dtype=torch.uint8, device=self.device)
-        self.h_slots, self.h_lens, self.h_pairs, self.h_tables = (
-            self._view(self.h_meta, n) for n in ("slots", "lens", "pairs", "tables"))
-        self.s_slots, self.s_lens, self.s_pairs, self.s_tables = (
-            self._view(self.d_meta, n) for n in ("slots", "lens", "pairs", "tables"))
-        self._ptr = {n: ctypes.c_void_p(self.h_meta.data_ptr() + self._layout[n][0]) for n in self._layout}
+        for name, dtype, shape in (("slots", torch.int64, (b,)), ("lens", torch.int32, (b,)),
+                                   ("pairs", torch.int32, (b, 2)), ("tables", torch.int32, (b, mb)),
+                                   ("q", torch.bfloat16, (b, num_q_heads, head_dim)),
+                                   ("k", torch.bfloat16, (b, num_kv_heads, head_dim)),
+                                   ("v", torch.bfloat16, (b, num_kv_heads, head_dim))):
+            nbytes_f = int(np.prod(shape)) * torch.empty((), dtype=dtype).element_size()
+            self._layout[name] = (off, dtype, shape, nbytes_f)
+            off += _align(nbytes_f)
+        self.stage_bytes = off
+        self.meta_bytes = self._layout["q"][0]
+        self.h_stage = [torch.zeros(off, dtype=torch.uint8).pin_memory() for _ in range(staging_sets)]
+        self.d_stage = torch.zeros(off, dtype=torch.uint8, device=self.device)
+        # device views the kernels (and a captured graph) read
+        (self.s_slots, self.s_lens, self.s_pairs, self.s_tables, self.s_q, self.s_k,
+         self.s_v) = (self._view(self.d_stage, n) for n in ("slots", "lens", "pairs", "tables", "q", "k", "v"))
         self._ncow = ctypes.c_int(0)
         self._ids = None
         self._ids_src = None
         self.graph = None
 
     def _view(self, buf, name):
-        off, dtype, count = self._layout[name]
-        t = buf[off:off + count * torch.empty((), dtype=dtype).element_size()].view(dtype)
-        if name == "pairs":
-            t = t.view(-1, 2)
-        elif name == "tables":
-            t = t.view(self.max_batch, self.max_blocks)
-        return t
+        off, dtype, shape, nbytes_f = self._layout[name]
+        return buf[off:off + nbytes_f].view(dtype).view(shape)
+
+    def staged(self, name, j=0):
+        """Host view of field ``name`` of pinned staging buffer ``j`` (fill
+        q / k / v here; the allocator fills the metadata)."""
+        return self._view(self.h_stage[j], name)
+
+    def _hptr(self, name, j):
+        return ctypes.c_void_p(self.h_stage[j].data_ptr() + self._layout[name][0])
 
     # ---------------------------------------------------------------- host
     def plan_append(self, seq_ids):
@@ -90,9 +100,9 @@ class PagedDecodeCache:
         tables, lens = self.alloc.block_tables(seq_ids, self.max_blocks)
         return slots, pairs, tables, lens
 
-    def host_step(self, seq_ids):
+    def host_step(self, seq_ids, j=0):
         """Allocator step for one new token per request (host only), written
-        straight into the pinned metadata buffer.  Returns the number of
+        straight into pinned staging buffer ``j``.  Returns the number of
         copy-on-write pairs.  ``seq_ids`` must hold max_batch requests."""
         if self._ids is None or self._ids_src is not seq_ids:
             self._ids = np.ascontiguousarray(np.asarray(seq_ids, dtype=np.int64))
@@ -101,19 +111,22 @@ class PagedDecodeCache:
         h = self.alloc._h
         ids = ctypes.c_void_p(self._ids.ctypes.data)
         b = self.max_batch
-        _check(lib.pa_alloc_append_batch(h, ids, b, 1, self._ptr["slots"], self._ptr["pairs"], b,
+        _check(lib.pa_alloc_append_batch(h, ids, b, 1, self._hptr("slots", j), self._hptr("pairs", j), b,
                                          ctypes.byref(self._ncow)), "pa_alloc_append_batch")
-        _check(lib.pa_alloc_block_tables(h, ids, b, self.max_blocks, self._ptr["tables"], self._ptr["lens"]),
-               "pa_alloc_block_tables")
+        _check(lib.pa_alloc_block_tables(h, ids, b, self.max_blocks, self._hptr("tables", j),
+                                         self._hptr("lens", j)), "pa_alloc_block_tables")
         return self._ncow.value
 
-    def upload(self):
-        """One host-to-device copy of the staged metadata (async, pinned)."""
-        self.d_meta.copy_(self.h_meta, non_blocking=True)
+    def upload(self, j=0, with_inputs=True):
+        """One host-to-device copy of staging buffer ``j`` (metadata, and the
+        q / k / v inputs unless ``with_inputs`` is false); async, pinned."""
+        n = self.stage_bytes if with_inputs else self.meta_bytes
+        self.d_stage[:n].copy_(self.h_stage[j][:n], non_blocking=True)
 
-    def capture(self, q, k_new, v_new, out):
-        """Record the device part of a step (cache write, decode, merge) on the
-        staged device metadata into a CUDA graph; replay it with ``replay``.
+    def capture(self, out):
+        """Record the device part of a step -- the new tokens' cache write
+        fused with the decode, and the merge -- on the staged device buffers
+        into a CUDA graph; replay it with ``replay``.
 
         Call after one ``host_step`` + ``upload`` so the staged slots are
         real: the eager warm-up run writes the step's own K/V, which the
@@ -121,16 +134,16 @@ class PagedDecodeCache:
         side = torch.cuda.Stream(device=self.device)
         side.wait_stream(torch.cuda.current_stream(self.device))
         with torch.cuda.stream(side):
-            self._device_step(q, k_new, v_new, out)
+            self._device_step(out)
         torch.cuda.current_stream(self.device).wait_stream(side)
         g = torch.cuda.CUDAGraph()
         with torch.cuda.graph(g):
-            self._device_step(q, k_new, v_new, out)
+            self._device_step(out)
         self.graph = g
         return g
 
-    def _device_step(self, q, k_new, v_new, out):
-        self.append_decode(q, k_new, v_new, out, self.s_slots, self.s_tables, self.s_lens)
+    def _device_step(self, out):
+        self.append_decode(self.s_q, self.s_k, self.s_v, out, self.s_slots, self.s_tables, self.s_lens)
 
     def replay(self, npairs):
         """Device part of a staged step: copy-on-write copies (if any), then the graph."""

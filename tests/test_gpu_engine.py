@@ -51,10 +51,7 @@ def test_graph_replayed_steps_match_oracle(schedule):
         a.free_seq(100)
         a.free_seq(101)
     ids = list(range(6))
-    q = torch.empty((6, hq, d), dtype=torch.bfloat16, device=dev)
-    k = torch.empty((6, hkv, d), dtype=torch.bfloat16, device=dev)
-    v = torch.empty_like(k)
-    out = torch.empty_like(q)
+    out = torch.empty((6, hq, d), dtype=torch.bfloat16, device=dev)
     scale = 1.0 / math.sqrt(d)
 
     def oracle_step(qh, kh, vh):
@@ -73,21 +70,22 @@ def test_graph_replayed_steps_match_oracle(schedule):
         npairs = cache.host_step(ids)
         slots, pairs, tables, lens, want = oracle_step(qh, kh, vh)
         # the allocator's staged output equals the oracle's
-        assert cache.h_slots.numpy().tolist() == list(slots)
+        assert cache.staged("slots").numpy().tolist() == list(slots)
         assert npairs == len(pairs)
-        assert [tuple(p) for p in cache.h_pairs[:npairs].numpy().tolist()] == [tuple(p) for p in pairs]
-        assert np.array_equal(cache.h_tables.numpy(), tables) and np.array_equal(cache.h_lens.numpy(), lens)
+        assert [tuple(p) for p in cache.staged("pairs")[:npairs].numpy().tolist()] == [tuple(p) for p in pairs]
+        assert np.array_equal(cache.staged("tables").numpy(), tables)
+        assert np.array_equal(cache.staged("lens").numpy(), lens)
         seen_cow += npairs
+        cache.staged("q").copy_(qh)
+        cache.staged("k").copy_(kh)
+        cache.staged("v").copy_(vh)
         cache.upload()
-        q.copy_(qh)
-        k.copy_(kh)
-        v.copy_(vh)
         if step == 0:
-            # record the device part on this step's staged metadata; the
-            # capture's warm-up already performs this step's copies + write
+            # record the device part on this step's staged data; the capture's
+            # warm-up already performs this step's copies and cache write
             if npairs:
                 pk.pa_copy_blocks(cache.pool, cache.s_pairs[:npairs])
-            cache.capture(q, k, v, out)
+            cache.capture(out)
         else:
             cache.replay(npairs)
         torch.cuda.synchronize()
