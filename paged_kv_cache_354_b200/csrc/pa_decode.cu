@@ -39,6 +39,7 @@ namespace pa {
 constexpr int kConsumerWarps = 4;
 constexpr int kThreads = (kConsumerWarps + 1) * 32;
 constexpr int kMaxGroup = 8;
+constexpr float kRescaleSlack = 8.f;  // log2 units: probabilities stay <= 256
 constexpr unsigned kFull = 0xffffffffu;
 
 enum Variant { kCudaCore = 1, kMma = 2 };
@@ -198,6 +199,11 @@ struct MmaConsumer {
         }
       }
     }
+    // The kept max m may lag the true running max by up to kRescaleSlack
+    // (log2 units): p = 2^(s - m) then stays <= 2^kRescaleSlack, which bf16 P
+    // and the fp32 sums hold with the same relative precision, and the final
+    // normalisation divides by a sum taken against the same m.  So the
+    // accumulators are rescaled only when some column's max grows past it.
     bool moved = false;
 #pragma unroll
     for (int nt = 0; nt < NT; ++nt)
@@ -206,10 +212,10 @@ struct MmaConsumer {
 #pragma unroll
         for (int off = 4; off < 32; off <<= 1)
           mx[nt][e] = fmaxf(mx[nt][e], __shfl_xor_sync(kFull, mx[nt][e], off));
+        moved |= mx[nt][e] > m[nt][e] + kRescaleSlack;  // also true while m = -inf
         mx[nt][e] = fmaxf(m[nt][e], mx[nt][e]);
-        moved |= mx[nt][e] > m[nt][e];
       }
-    // rescale only when some column's running max moved (warp-uniform test)
+    // rescale only when some column's kept max is too low (warp-uniform test)
     if (__any_sync(kFull, moved)) {
 #pragma unroll
       for (int nt = 0; nt < NT; ++nt)
