@@ -166,11 +166,17 @@ struct MmaConsumer {
     const int mat = lane >> 3;
     const int r8 = lane & 7;
     // ---- S^T = K Q^T : rows = tokens of the block, cols = (token, head)
+    // two independent accumulation chains over the head dim (even / odd
+    // 16-dim steps), summed at the end: half the dependent MMA latency
     float s[kTT][NT][4];
 #pragma unroll
     for (int mt = 0; mt < kTT; ++mt) {
+      float s2[NT][4];
 #pragma unroll
-      for (int nt = 0; nt < NT; ++nt) s[mt][nt][0] = s[mt][nt][1] = s[mt][nt][2] = s[mt][nt][3] = 0.f;
+      for (int nt = 0; nt < NT; ++nt) {
+        s[mt][nt][0] = s[mt][nt][1] = s[mt][nt][2] = s[mt][nt][3] = 0.f;
+        s2[nt][0] = s2[nt][1] = s2[nt][2] = s2[nt][3] = 0.f;
+      }
       const int tok = 16 * mt + ((mat & 1) << 3) + r8;
 #pragma unroll
       for (int ks = 0; ks < kDT; ++ks) {
@@ -179,8 +185,15 @@ struct MmaConsumer {
         uint32_t a0, a1, a2, a3;
         ldsm_x4(addr, a0, a1, a2, a3);
 #pragma unroll
-        for (int nt = 0; nt < NT; ++nt) mma_bf16_16816(s[mt][nt], a0, a1, a2, a3, qb[nt][ks][0], qb[nt][ks][1]);
+        for (int nt = 0; nt < NT; ++nt) {
+          if (ks & 1) mma_bf16_16816(s2[nt], a0, a1, a2, a3, qb[nt][ks][0], qb[nt][ks][1]);
+          else mma_bf16_16816(s[mt][nt], a0, a1, a2, a3, qb[nt][ks][0], qb[nt][ks][1]);
+        }
       }
+#pragma unroll
+      for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+        for (int e = 0; e < 4; ++e) s[mt][nt][e] += s2[nt][e];
     }
     // ---- scale, mask positions each column may not see, column max
     float mx[NT][2];
