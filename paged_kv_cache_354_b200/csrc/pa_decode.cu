@@ -195,7 +195,7 @@ struct MmaConsumer {
 #pragma unroll
         for (int e = 0; e < 4; ++e) s[mt][nt][e] += s2[nt][e];
     }
-    // ---- scale, mask positions each column may not see, column max
+    // ---- scale, mask positions each column may not see, local max
     float mx[NT][2];
 #pragma unroll
     for (int nt = 0; nt < NT; ++nt) mx[nt][0] = mx[nt][1] = -INFINITY;
@@ -215,33 +215,32 @@ struct MmaConsumer {
     // The kept max m may lag the true running max by up to kRescaleSlack
     // (log2 units): p = 2^(s - m) then stays <= 2^kRescaleSlack, which bf16 P
     // and the fp32 sums hold with the same relative precision, and the final
-    // normalisation divides by a sum taken against the same m.  So the
-    // accumulators are rescaled only when some column's max grows past it.
-    bool moved = false;
+    // normalisation divides by a sum taken against the same m.  Each thread
+    // checks its own logits against that bound; only when one exceeds it
+    // (always on a column's first visible block) does the warp form the exact
+    // column max with shuffles and rescale the accumulators.
+    bool over = false;
 #pragma unroll
     for (int nt = 0; nt < NT; ++nt)
 #pragma unroll
-      for (int e = 0; e < 2; ++e) {
-#pragma unroll
-        for (int off = 4; off < 32; off <<= 1)
-          mx[nt][e] = fmaxf(mx[nt][e], __shfl_xor_sync(kFull, mx[nt][e], off));
-        moved |= mx[nt][e] > m[nt][e] + kRescaleSlack;  // also true while m = -inf
-        mx[nt][e] = fmaxf(m[nt][e], mx[nt][e]);
-      }
-    // rescale only when some column's kept max is too low (warp-uniform test)
-    if (__any_sync(kFull, moved)) {
+      for (int e = 0; e < 2; ++e) over |= mx[nt][e] > m[nt][e] + kRescaleSlack;  // true while m = -inf
+    if (__any_sync(kFull, over)) {
 #pragma unroll
       for (int nt = 0; nt < NT; ++nt)
 #pragma unroll
         for (int e = 0; e < 2; ++e) {
-          const float a = (m[nt][e] == -INFINITY) ? 0.f : exp2f(m[nt][e] - mx[nt][e]);
+#pragma unroll
+          for (int off = 4; off < 32; off <<= 1)
+            mx[nt][e] = fmaxf(mx[nt][e], __shfl_xor_sync(kFull, mx[nt][e], off));
+          const float mnew = fmaxf(m[nt][e], mx[nt][e]);
+          const float a = (m[nt][e] == -INFINITY) ? 0.f : exp2f(m[nt][e] - mnew);
 #pragma unroll
           for (int dt = 0; dt < kDT; ++dt) {
             o[dt][nt][e] *= a;
             o[dt][nt][e + 2] *= a;
           }
           l[nt][e] *= a;
-          m[nt][e] = mx[nt][e];
+          m[nt][e] = mnew;
         }
     }
     // ---- P (bf16) -> P^T fragments; O^T += V^T P^T.  A column that has seen
