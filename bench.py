@@ -547,7 +547,9 @@ def study_memory_waste():
 def study_page_table(iters=30):
     """pa_decode on the workload's scattered block tables vs on identity
     tables (each request's blocks physically consecutive, same lengths and
-    pool format): the cost the block-table indirection adds to the kernel
+    pool format), and vs pa_decode_contiguous on a contiguous reservation per
+    request (no block table at all; the quiz page's "Naive contiguous
+    allocation"): the cost the block-table indirection adds to the kernel
     (quiz page, comparison table row "Kernel overhead": small, <5%)."""
     import torch
 
@@ -593,11 +595,42 @@ def study_page_table(iters=30):
             res[layout] = (us, nbytes / us / 1e3)
             del cache
             torch.cuda.empty_cache()
+        # the same lengths in one contiguous run per request, 16-row tiles
+        lens_c = np.asarray(p.seq_lens, dtype=np.int32)
+        max_len = -(-int(lens_c.max()) // 16) * 16
+        gen = torch.Generator(device=dev)
+        gen.manual_seed(workloads.seed_of(name) + 1)
+        kv = torch.randn((len(lens_c), 2, s.num_kv_heads, max_len, s.head_dim), generator=gen, device=dev,
+                         dtype=torch.bfloat16)
+        q = torch.randn((len(lens_c), s.num_q_heads, s.head_dim), generator=gen, device=dev).bfloat16()
+        out = torch.empty_like(q)
+        d_l = torch.as_tensor(lens_c, device=dev)
+        ws = torch.empty(pk.pa_decode_contiguous_workspace_size(len(lens_c), s.num_q_heads, s.num_kv_heads,
+                                                                 s.head_dim, max_len), dtype=torch.uint8, device=dev)
+        scale = 1.0 / float(np.sqrt(s.head_dim))
+        for _ in range(3):
+            pk.pa_decode_contiguous(out, q, kv, d_l, scale, ws)
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        for _ in range(iters):
+            pk.pa_decode_contiguous(out, q, kv, d_l, scale, ws)
+        e1.record()
+        torch.cuda.synchronize()
+        us = e0.elapsed_time(e1) / iters * 1e3
+        kv_bytes = int(lens_c.astype(np.int64).sum()) * 2 * s.num_kv_heads * s.head_dim * 2
+        res["contiguous"] = (us, (kv_bytes + 2 * q.numel() * 2 + 4 * len(lens_c)) / us / 1e3)
+        del kv
+        torch.cuda.empty_cache()
         print(json.dumps({
             "study": "page_table_overhead", "workload": name,
             "scattered_us": round(res["scattered"][0], 2), "identity_us": round(res["identity"][0], 2),
+            "contiguous_us": round(res["contiguous"][0], 2),
             "scattered_gbs": round(res["scattered"][1], 1), "identity_gbs": round(res["identity"][1], 1),
+            "contiguous_gbs": round(res["contiguous"][1], 1),
             "overhead_frac": round(res["scattered"][0] / res["identity"][0] - 1, 4),
+            "overhead_vs_contiguous_frac": round(res["scattered"][0] / res["contiguous"][0] - 1, 4),
+            "paged_block_size": s.block_size, "contiguous_tile_rows": 16,
             "iters": iters}), flush=True)
     assert pk.pa_device_error() == 0
 

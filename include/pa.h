@@ -285,6 +285,36 @@ int pa_decode_multi(pa_bf16* out, const pa_bf16* q, const pa_bf16* kv_pool,
                     int block_size, int num_blocks, int max_blocks_per_seq, int max_seq_len,
                     float scale, void* workspace, size_t workspace_bytes, void* stream);
 
+/* --------------------------------------------------------------------------
+ * pa_decode_contiguous -- the same attention over a contiguous cache.
+ *
+ * The baseline paging replaces: the quiz page's comparison table, column
+ * "Naive contiguous allocation" (row "Reservation per request": a buffer
+ * sized for the maximum context; row "Kernel overhead": none).  Each request
+ * owns one reserved run of max_len positions, keys then values:
+ *
+ *   kv_cache : device bf16 [batch][2][num_kv_heads][max_len][head_dim]
+ *              (index 0 on the second axis keys, 1 values)
+ *
+ * and out[b, j] is the softmax(q K^T scale) V of pa_decode over positions
+ * [0, seq_lens[b]) of that run -- no block table.  It runs pa_decode's
+ * balanced kernel and arithmetic with the table lookup replaced by direct
+ * 16-row tile addressing, so at equal lengths the two layouts give the same
+ * result bit for bit and their timing difference is the cost of paging.
+ * max_len must be a positive multiple of 16; seq_lens[b] > max_len is
+ * flagged (PA_DEVERR_SEQ_LEN) and clamped.  variant: PA_DECODE_AUTO,
+ * PA_DECODE_CUDA_CORE (group 1, 2, 4) or PA_DECODE_MMA.  batch <= 4096.
+ * Workspace from pa_decode_contiguous_workspace_size (never 0 bytes).
+ * Other arguments as pa_decode.
+ * ------------------------------------------------------------------------ */
+int pa_decode_contiguous_workspace_size(int batch, int num_q_heads, int num_kv_heads, int head_dim,
+                                        int max_len, size_t* bytes_out);
+
+int pa_decode_contiguous(pa_bf16* out, const pa_bf16* q, const pa_bf16* kv_cache,
+                         const int32_t* seq_lens, int batch, int num_q_heads, int num_kv_heads,
+                         int head_dim, int max_len, float scale, void* workspace,
+                         size_t workspace_bytes, int variant, void* stream);
+
 /* Self-test of the bounded pipeline wait used by the kernels: one CTA waits
  * on a barrier phase that nothing completes, for at most limit_ns, then
  * returns.  Expect PA_DEVERR_WAIT_TIMEOUT in pa_device_error() afterwards.

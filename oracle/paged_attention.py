@@ -128,6 +128,36 @@ def decode_one(query_vec, kv_pool, block_table_row, seq_len, kv_head, scale):
     return weights @ values[:, kv_head, :]
 
 
+def decode_contiguous(query, kv_cache, seq_lens, scale):
+    """Single-token decode over a contiguous per-request cache, in float64.
+
+    The layout paging replaces: the quiz page's comparison table, column
+    "Naive contiguous allocation", reserves a buffer of the maximum context
+    for every request; "Paged attention in LLMs", section "Why the memory
+    gets wasted", reserves that maximum up front in one unbroken run.  Here
+    request b's run is ``kv_cache[b]`` = [2, Hkv, max_len, D] (keys, then
+    values) and positions [0, L_b) of it hold the request's cache.  The
+    attention is the same textbook one as ``decode``, with no table.
+
+    query : float64 [B, Hq, D]; kv_cache : float64 [B, 2, Hkv, max_len, D]
+    seq_lens : int [B]; returns float64 [B, Hq, D] (0 for L_b = 0).
+    """
+    batch, num_q_heads, head_dim = query.shape
+    num_kv_heads = kv_cache.shape[2]
+    group = num_q_heads // num_kv_heads
+    out = np.zeros((batch, num_q_heads, head_dim), dtype=np.float64)
+    for b in range(batch):
+        seq_len = int(seq_lens[b])
+        for j in range(num_q_heads if seq_len > 0 else 0):
+            keys = kv_cache[b, 0, j // group, :seq_len]
+            values = kv_cache[b, 1, j // group, :seq_len]
+            logits = scale * (keys @ query[b, j])
+            weights = np.exp(logits - logits.max())
+            weights /= weights.sum()
+            out[b, j] = weights @ values
+    return out
+
+
 def decode_multi(query, kv_pool, block_tables, seq_lens, scale):
     """T query tokens per request, each attending causally (float64).
 

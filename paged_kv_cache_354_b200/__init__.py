@@ -11,6 +11,7 @@ bf16 tensors are ``torch.bfloat16``; shapes follow ``include/pa.h``:
     kv_pool      [num_blocks, 2, num_kv_heads, block_size, head_dim]
     q, out       [batch, num_q_heads, head_dim]
     key, value   [num_tokens, num_kv_heads, head_dim]
+    kv_cache     [batch, 2, num_kv_heads, max_len, head_dim]  (contiguous decode)
     block_tables int32 [batch, max_blocks_per_seq]; seq_lens int32 [batch]
     slot_mapping int64 [num_tokens]; block_pairs int32 [num_pairs, 2]
 """
@@ -66,6 +67,8 @@ _SIGNATURES = {
     "pa_decode_multi_workspace_size": (_I, [_I, _I, _I, _I, _I, _I, _I, _P]),
     "pa_decode_multi": (_I, [_P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _I, _I, _I, _c.c_float, _P, _SZ,
                              _P]),
+    "pa_decode_contiguous_workspace_size": (_I, [_I, _I, _I, _I, _I, _P]),
+    "pa_decode_contiguous": (_I, [_P, _P, _P, _P, _I, _I, _I, _I, _I, _c.c_float, _P, _SZ, _I, _P]),
     "pa_selftest_wait_timeout": (_I, [_I64, _P]),
     "pa_alloc_create": (_I, [_I, _I, _P, _P]),
     "pa_alloc_destroy": (_I, [_P]),
@@ -247,6 +250,32 @@ def pa_decode_multi(out, q, kv_pool, block_tables, seq_lens, max_seq_len, scale,
     _check(lib.pa_decode_multi(_ptr(out), _ptr(q), _ptr(kv_pool), _ptr(block_tables), _ptr(seq_lens), b, t, hq,
                                hkv, d, bs, nb, block_tables.shape[1], int(max_seq_len), float(scale),
                                _ptr(workspace), workspace.numel(), _stream(stream)), "pa_decode_multi")
+
+
+def pa_decode_contiguous_workspace_size(batch, num_q_heads, num_kv_heads, head_dim, max_len):
+    nbytes = ctypes.c_size_t(0)
+    _check(lib.pa_decode_contiguous_workspace_size(batch, num_q_heads, num_kv_heads, head_dim, max_len,
+                                                   ctypes.byref(nbytes)), "pa_decode_contiguous_workspace_size")
+    return nbytes.value
+
+
+def pa_decode_contiguous(out, q, kv_cache, seq_lens, scale, workspace, variant=PA_DECODE_AUTO, stream=None):
+    """Decode over a contiguous per-request cache kv_cache bf16
+    [B, 2, Hkv, max_len, D] (no block table); writes ``out`` in place."""
+    import torch
+
+    _require(out, torch.bfloat16, "out")
+    _require(q, torch.bfloat16, "q")
+    _require(kv_cache, torch.bfloat16, "kv_cache")
+    _require(seq_lens, torch.int32, "seq_lens")
+    _require(workspace, torch.uint8, "workspace")
+    b, two, hkv, max_len, d = kv_cache.shape
+    bq, hq, dq = q.shape
+    if two != 2 or out.shape != q.shape or dq != d or bq != b or seq_lens.shape != (b,):
+        raise ValueError("pa_decode_contiguous: shape mismatch")
+    _check(lib.pa_decode_contiguous(_ptr(out), _ptr(q), _ptr(kv_cache), _ptr(seq_lens), b, hq, hkv, d, max_len,
+                                    float(scale), _ptr(workspace), workspace.numel(), int(variant),
+                                    _stream(stream)), "pa_decode_contiguous")
 
 
 PA_NOALLOC_SCRATCH_BYTES = 16 * 1024 * 1024

@@ -845,7 +845,13 @@ __device__ __forceinline__ void consumer_bar() {
   asm volatile("bar.sync 1, %0;" ::"n"(kConsumerWarps * 32) : "memory");
 }
 
-template <int D, int BS, int VAR, int G, int NT>
+// Where a (request, KV head, block) tile lives.  kPaged: the pool
+// [NB][2][Hkv][bs][D] through the block table.  kContiguous: one reserved
+// run per request, [B][2][Hkv][max_len][D], block k being rows
+// [k bs, (k+1) bs) -- no table; the naive layout paging replaces.
+enum Layout { kPaged = 0, kContiguous = 1 };
+
+template <int D, int BS, int VAR, int G, int NT, int LAYOUT = kPaged>
 __global__ void __launch_bounds__(kThreads, kStreamCtasPerSm)
     paged_decode_stream_kernel(const __grid_constant__ CUtensorMap kv_map, const DecodeArgs a,
                                int batch) {
@@ -900,19 +906,21 @@ __global__ void __launch_bounds__(kThreads, kStreamCtasPerSm)
     while (u < u_end && !stop) {
       const int nb = prefix[b + 1] - prefix[b];
       const int cnt = static_cast<int>(min(static_cast<long long>(nb - k), u_end - u));
-      const int32_t* trow = a.block_tables + static_cast<size_t>(b) * a.max_blocks_per_seq + k;
       for (int base = 0; base < cnt && !stop; base += 32) {
         int phys = 0;
-        if (base + lane < cnt) {
-          phys = __ldg(trow + base + lane);
-          if (static_cast<unsigned>(phys) >= static_cast<unsigned>(a.num_blocks)) {
-            flag_error(a.err, PA_DEVERR_BLOCK_ID);
-            phys = 0;  // read a valid block instead; the result is flagged as wrong
+        if constexpr (LAYOUT == kPaged) {
+          const int32_t* trow = a.block_tables + static_cast<size_t>(b) * a.max_blocks_per_seq + k;
+          if (base + lane < cnt) {
+            phys = __ldg(trow + base + lane);
+            if (static_cast<unsigned>(phys) >= static_cast<unsigned>(a.num_blocks)) {
+              flag_error(a.err, PA_DEVERR_BLOCK_ID);
+              phys = 0;  // read a valid block instead; the result is flagged as wrong
+            }
           }
         }
         const int n32 = min(32, cnt - base);
         for (int j = 0; j < n32; ++j) {
-          const int pb = __shfl_sync(kFull, phys, j);
+          const int pb = (LAYOUT == kPaged) ? __shfl_sync(kFull, phys, j) : 0;
           int failed = 0;
           if (lane == 0) {
             const int ii = i + base + j;
@@ -926,9 +934,15 @@ __global__ void __launch_bounds__(kThreads, kStreamCtasPerSm)
               const uint32_t fb = bar_full + 8 * s;
               mbar_arrive_expect_tx(fb, geo::kStageBytes);
               const uint32_t dst = sbase + s * geo::kStageBytes;
+              if constexpr (LAYOUT == kPaged) {
 #pragma unroll
-              for (int x = 0; x < geo::kRegions; ++x)
-                tma_load_3d(dst + x * geo::kRegionBytes, &kv_map, fb, x * 64, h * BS, 2 * pb);
+                for (int x = 0; x < geo::kRegions; ++x)
+                  tma_load_3d(dst + x * geo::kRegionBytes, &kv_map, fb, x * 64, h * BS, 2 * pb);
+              } else {  // rows of block k + base + j of request b, head h; keys then values
+#pragma unroll
+                for (int x = 0; x < geo::kRegions; ++x)
+                  tma_load_4d(dst + x * geo::kRegionBytes, &kv_map, fb, x * 64, (k + base + j) * BS, h, 2 * b);
+              }
               last_round[s] = round;
             }
           }
@@ -1383,11 +1397,11 @@ static int launch_main(const CUtensorMap& map, const DecodeArgs& a, int batch, c
   return PA_OK;
 }
 
-template <int D, int BS, int VAR, int G, int NT = 1>
+template <int D, int BS, int VAR, int G, int NT = 1, int LAYOUT = kPaged>
 static int launch_stream(const CUtensorMap& map, const DecodeArgs& a, int batch, int ctas,
                          cudaStream_t st) {
   using sm = StreamSmem<D, BS, G, NT>;
-  auto kern = paged_decode_stream_kernel<D, BS, VAR, G, NT>;
+  auto kern = paged_decode_stream_kernel<D, BS, VAR, G, NT, LAYOUT>;
   const int smem = sm::dynamic_bytes(batch, a.cols);
   int rc = set_smem_attr(reinterpret_cast<const void*>(kern), smem);
   if (rc != PA_OK) return rc;
@@ -1542,6 +1556,102 @@ static int decode_impl(pa_bf16* out, const pa_bf16* q, const pa_bf16* kv_pool,
   return dispatch<128, 32>(map, a, batch, variant, plan, st);
 }
 
+// Decode over a contiguous per-request cache [B][2][Hkv][max_len][D]: the
+// balanced kernel with the table gather replaced by direct row addressing
+// (16-row tiles), so the two layouts run the same schedule and arithmetic.
+constexpr int kContiguousTile = 16;
+
+template <int D>
+static int dispatch_contiguous(const CUtensorMap& map, const DecodeArgs& a, int batch, int variant,
+                               int ctas, cudaStream_t st) {
+  constexpr int T = kContiguousTile;
+  if (variant == kMma) return launch_stream<D, T, kMma, 0, 1, kContiguous>(map, a, batch, ctas, st);
+  switch (a.group) {
+    case 1: return launch_stream<D, T, kCudaCore, 1, 1, kContiguous>(map, a, batch, ctas, st);
+    case 2: return launch_stream<D, T, kCudaCore, 2, 1, kContiguous>(map, a, batch, ctas, st);
+    case 4: return launch_stream<D, T, kCudaCore, 4, 1, kContiguous>(map, a, batch, ctas, st);
+    default:
+      return fail(PA_ERR_UNSUPPORTED, "pa_decode_contiguous: CUDA-core variant has no group size %d", a.group);
+  }
+}
+
+static int contiguous_plan(int batch, int hq, int hkv, int d, int max_len, Plan* plan) {
+  int rc = check_shape(batch, hq, hkv, d, kContiguousTile, max_len);
+  if (rc != PA_OK) return rc;
+  if (max_len <= 0 || max_len % kContiguousTile != 0)
+    return fail(PA_ERR_INVALID, "pa_decode_contiguous: max_len %d not a positive multiple of %d", max_len,
+                kContiguousTile);
+  return make_plan(batch, hq, hkv, d, kContiguousTile, max_len, kForceBalanced, plan);
+}
+
+static int decode_contiguous_impl(pa_bf16* out, const pa_bf16* q, const pa_bf16* kv_cache,
+                                  const int32_t* seq_lens, int batch, int hq, int hkv, int d,
+                                  int max_len, float scale, void* workspace, size_t ws_bytes,
+                                  int variant, void* stream) {
+  Plan plan;
+  int rc = contiguous_plan(batch, hq, hkv, d, max_len, &plan);
+  if (rc != PA_OK) return rc;
+  if (!std::isfinite(scale)) return fail(PA_ERR_INVALID, "pa_decode_contiguous: scale is not finite");
+  if (batch == 0) return PA_OK;
+  if (!out || !q || !kv_cache || !seq_lens) return fail(PA_ERR_INVALID, "pa_decode_contiguous: NULL pointer");
+  auto a16 = [](const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; };
+  if (!a16(out) || !a16(q) || !a16(kv_cache) || (reinterpret_cast<uintptr_t>(seq_lens) & 3u))
+    return fail(PA_ERR_INVALID, "pa_decode_contiguous: misaligned pointer");
+  const int group = hq / hkv;
+  if (variant == PA_DECODE_AUTO) variant = group >= 4 ? kMma : kCudaCore;
+  if (variant != kCudaCore && variant != kMma)
+    return fail(PA_ERR_INVALID, "pa_decode_contiguous: unknown variant %d", variant);
+  if (variant == kCudaCore && group != 1 && group != 2 && group != 4)
+    return fail(PA_ERR_UNSUPPORTED, "pa_decode_contiguous: CUDA-core variant has no group size %d", group);
+  if (workspace == nullptr || ws_bytes < plan.bytes)
+    return fail(PA_ERR_INVALID, "pa_decode_contiguous: workspace of %zu bytes needed, %zu given", plan.bytes,
+                workspace ? ws_bytes : static_cast<size_t>(0));
+  if (reinterpret_cast<uintptr_t>(workspace) & 255u)
+    return fail(PA_ERR_INVALID, "pa_decode_contiguous: workspace not 256-byte aligned");
+  int32_t* err = device_error_word();
+  if (err == nullptr) return PA_ERR_CUDA;
+
+  // TMA view: x = head dim, y = row (position), z = KV head, w = 2*request +
+  // (0 keys | 1 values); a box of 2 along w brings a tile's keys and values.
+  alignas(64) CUtensorMap map;
+  const uint64_t dims[4] = {static_cast<uint64_t>(d), static_cast<uint64_t>(max_len),
+                            static_cast<uint64_t>(hkv), 2ull * static_cast<uint64_t>(batch)};
+  const uint64_t strides[3] = {static_cast<uint64_t>(d) * 2, static_cast<uint64_t>(max_len) * d * 2,
+                               static_cast<uint64_t>(hkv) * max_len * d * 2};
+  const uint32_t box[4] = {64u, static_cast<uint32_t>(kContiguousTile), 1u, 2u};
+  rc = encode_tensor_map(&map, 4, const_cast<pa_bf16*>(kv_cache), dims, strides, box, 1);
+  if (rc != PA_OK) return rc;
+
+  DecodeArgs a{};
+  a.out = reinterpret_cast<__nv_bfloat16*>(out);
+  a.q = reinterpret_cast<const __nv_bfloat16*>(q);
+  a.block_tables = nullptr;
+  a.seq_lens = seq_lens;
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  a.part_o = reinterpret_cast<float*>(ws);
+  a.part_m = reinterpret_cast<float*>(ws + plan.off_m);
+  a.part_l = reinterpret_cast<float*>(ws + plan.off_l);
+  a.err = err;
+  a.num_q_heads = hq;
+  a.num_kv_heads = hkv;
+  a.group = group;
+  a.num_blocks = 0;
+  a.max_blocks_per_seq = max_len / kContiguousTile;  // lengths above max_len are flagged and clamped
+  a.part_blocks = a.max_blocks_per_seq;
+  a.max_parts = 1;
+  a.scale_log2 = scale * 1.4426950408889634f;
+  a.stream_prefix = reinterpret_cast<int*>(ws + plan.off_prefix);
+  a.qtok = 1;
+  a.cols = group;
+  a.new_k = nullptr;
+  a.new_v = nullptr;
+  a.new_slots = nullptr;
+  a.pool_w = nullptr;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (d == 64) return dispatch_contiguous<64>(map, a, batch, variant, plan.ctas, st);
+  return dispatch_contiguous<128>(map, a, batch, variant, plan.ctas, st);
+}
+
 }  // namespace pa
 
 extern "C" {
@@ -1633,6 +1743,24 @@ int pa_decode_ex(pa_bf16* out, const pa_bf16* q, const pa_bf16* kv_pool,
                          num_kv_heads, head_dim, block_size, num_blocks, max_blocks_per_seq,
                          max_seq_len, scale, workspace, workspace_bytes, variant, partition_tokens,
                          stream);
+}
+
+int pa_decode_contiguous_workspace_size(int batch, int num_q_heads, int num_kv_heads, int head_dim,
+                                        int max_len, size_t* bytes_out) {
+  using namespace pa;
+  if (bytes_out == nullptr) return fail(PA_ERR_INVALID, "pa_decode_contiguous_workspace_size: NULL bytes_out");
+  Plan plan;
+  int rc = contiguous_plan(batch, num_q_heads, num_kv_heads, head_dim, max_len, &plan);
+  if (rc != PA_OK) return rc;
+  *bytes_out = plan.bytes;
+  return PA_OK;
+}
+
+int pa_decode_contiguous(pa_bf16* out, const pa_bf16* q, const pa_bf16* kv_cache, const int32_t* seq_lens,
+                         int batch, int num_q_heads, int num_kv_heads, int head_dim, int max_len,
+                         float scale, void* workspace, size_t workspace_bytes, int variant, void* stream) {
+  return pa::decode_contiguous_impl(out, q, kv_cache, seq_lens, batch, num_q_heads, num_kv_heads, head_dim,
+                                    max_len, scale, workspace, workspace_bytes, variant, stream);
 }
 
 }  // extern "C"

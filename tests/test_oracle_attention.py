@@ -15,6 +15,8 @@ product attention".  These pins tie the oracle to things other than itself:
   positions give logistic weights; constant V per KV head reveals the
   query-head -> KV-head mapping;
 * invariance under any permutation of the physical blocks;
+* the contiguous-reservation decode equals the paged decode on the same
+  sequences (and torch SDPA);
 * mutation tests: plausible single mistakes planted in a copy of the oracle
   (on the CPU) must each fail at least one pin.
 """
@@ -230,6 +232,43 @@ def pin_multi_short_request(m):
     np.testing.assert_allclose(got[0, 3], m.decode(qm[:, 3], pool, table, np.array([2]), 0.5)[0], atol=0)
 
 
+def contiguous_cache(ks, vs, max_len, fill=np.nan):
+    """[B, 2, Hkv, max_len, D] reservation per request (library ops only);
+    positions past each request's length hold ``fill``."""
+    hkv, d = ks[0].shape[1:]
+    cache = np.full((len(ks), 2, hkv, max_len, d), fill)
+    for b, (k, v) in enumerate(zip(ks, vs)):
+        cache[b, 0, :, :k.shape[0]] = k.transpose(1, 0, 2)
+        cache[b, 1, :, :v.shape[0]] = v.transpose(1, 0, 2)
+    return cache
+
+
+def pin_contiguous_matches_paged(m):
+    """The contiguous reservation and the paged pool hold the same sequence,
+    so decode over either gives the same output (the reservation's unused
+    tail, NaN here, is never read)."""
+    rng = np.random.default_rng(15)
+    lens = [1, 17, 40, 0, 33]
+    q, ks, vs, pool, table = random_case(rng, lens, 8, 2, 16, 4)
+    cache = contiguous_cache(ks, vs, 48)
+    got = m.decode_contiguous(q, cache, np.array(lens), 0.3)
+    want = m.decode(q, pool, table, np.array(lens), 0.3)
+    np.testing.assert_allclose(got, want, rtol=0, atol=1e-12)
+    assert np.array_equal(got[3], np.zeros((8, 16)))
+
+
+def pin_contiguous_sdpa(m):
+    """Against torch SDPA (fp64) on the request's keys and values."""
+    rng = np.random.default_rng(16)
+    lens, hq, hkv, d = [5, 64, 23], 12, 3, 32
+    ks = [rng.standard_normal((n, hkv, d)) for n in lens]
+    vs = [rng.standard_normal((n, hkv, d)) for n in lens]
+    q = rng.standard_normal((len(lens), hq, d))
+    got = m.decode_contiguous(q, contiguous_cache(ks, vs, 64), np.array(lens), 0.2)
+    for b in range(len(lens)):
+        np.testing.assert_allclose(got[b], sdpa_reference(q[b], ks[b], vs[b], 0.2), rtol=0, atol=1e-12)
+
+
 DECODE_PINS = [
     pin_gather_is_contiguous,
     pin_sdpa,
@@ -243,6 +282,8 @@ DECODE_PINS = [
     pin_multi_reduces_to_decode,
     pin_multi_causal_sdpa,
     pin_multi_short_request,
+    pin_contiguous_matches_paged,
+    pin_contiguous_sdpa,
 ]
 
 
@@ -266,6 +307,11 @@ MUTATIONS = {
     "keys_for_values": ("out[b, j] = weights @ values[:, h, :]", "out[b, j] = weights @ keys[:, h, :]"),
     "off_by_one_length": ("pos = np.arange(seq_len)", "pos = np.arange(1, seq_len + 1)"),
     "multi_not_causal": ("visible = int(seq_lens[b]) - tokens + t + 1", "visible = int(seq_lens[b])"),
+    "contiguous_k_v_swapped": ("keys = kv_cache[b, 0, j // group", "keys = kv_cache[b, 1, j // group"),
+    "contiguous_reads_past_length": ("keys = kv_cache[b, 0, j // group, :seq_len]",
+                                     "keys = kv_cache[b, 0, j // group, :seq_len + 1]"),
+    "contiguous_gqa_modulo": ("values = kv_cache[b, 1, j // group, :seq_len]",
+                              "values = kv_cache[b, 1, j % num_kv_heads, :seq_len]"),
     "multi_off_by_one": ("visible = int(seq_lens[b]) - tokens + t + 1", "visible = int(seq_lens[b]) - tokens + t"),
 }
 
