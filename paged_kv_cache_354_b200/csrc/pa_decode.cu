@@ -161,8 +161,14 @@ struct MmaConsumer {
     }
   }
 
-  // sb: staged block; pos0: position of its row 0 in the request.
-  __device__ __forceinline__ void step(uint32_t sb, int pos0, float scale_log2, int lane) {
+  // sb: staged block; pos0: position of its row 0 in the request; the
+  // stage goes back to the producer (arrive on empty_bar) once this warp has
+  // read it.  With one 16-token tile per block and one 8-column tile, V^T is
+  // read into registers right after S^T = K Q^T, so the stage is free for the
+  // next TMA load while the softmax and O^T += V^T P^T run (wider tiles keep
+  // V^T in shared memory: the extra 32 registers would spill).
+  __device__ __forceinline__ void step(uint32_t sb, int pos0, float scale_log2, int lane,
+                                       uint32_t empty_bar) {
     const int mat = lane >> 3;
     const int r8 = lane & 7;
     // ---- S^T = K Q^T : rows = tokens of the block, cols = (token, head)
@@ -194,6 +200,19 @@ struct MmaConsumer {
       for (int nt = 0; nt < NT; ++nt)
 #pragma unroll
         for (int e = 0; e < 4; ++e) s[mt][nt][e] += s2[nt][e];
+    }
+    constexpr bool kEarly = (kTT == 1 && NT == 1);
+    uint32_t vf[kEarly ? kDT : 1][4];
+    if constexpr (kEarly) {
+      const int row = BS + ((mat >> 1) << 3) + r8;
+#pragma unroll
+      for (int dt = 0; dt < kDT; ++dt) {
+        const int chunk = (2 * (dt & 3) + (mat & 1)) ^ r8;
+        ldsm_x4_trans(sb + (dt >> 2) * geo::kRegionBytes + row * 128 + chunk * 16, vf[dt][0], vf[dt][1],
+                      vf[dt][2], vf[dt][3]);
+      }
+      __syncwarp();
+      if (lane == 0) mbar_arrive(empty_bar);
     }
     // ---- scale, mask positions each column may not see, local max
     float mx[NT][2];
@@ -262,16 +281,28 @@ struct MmaConsumer {
         b0[nt] = movmatrix_trans(pa);
         b1[nt] = movmatrix_trans(pb);
       }
-      const int row = BS + 16 * mt + ((mat >> 1) << 3) + r8;
+      if constexpr (kEarly) {
 #pragma unroll
-      for (int dt = 0; dt < kDT; ++dt) {
-        const int chunk = (2 * (dt & 3) + (mat & 1)) ^ r8;
-        const uint32_t addr = sb + (dt >> 2) * geo::kRegionBytes + row * 128 + chunk * 16;
-        uint32_t a0, a1, a2, a3;
-        ldsm_x4_trans(addr, a0, a1, a2, a3);
+        for (int dt = 0; dt < kDT; ++dt)
 #pragma unroll
-        for (int nt = 0; nt < NT; ++nt) mma_bf16_16816(o[dt][nt], a0, a1, a2, a3, b0[nt], b1[nt]);
+          for (int nt = 0; nt < NT; ++nt)
+            mma_bf16_16816(o[dt][nt], vf[dt][0], vf[dt][1], vf[dt][2], vf[dt][3], b0[nt], b1[nt]);
+      } else {
+        const int row = BS + 16 * mt + ((mat >> 1) << 3) + r8;
+#pragma unroll
+        for (int dt = 0; dt < kDT; ++dt) {
+          const int chunk = (2 * (dt & 3) + (mat & 1)) ^ r8;
+          const uint32_t addr = sb + (dt >> 2) * geo::kRegionBytes + row * 128 + chunk * 16;
+          uint32_t a0, a1, a2, a3;
+          ldsm_x4_trans(addr, a0, a1, a2, a3);
+#pragma unroll
+          for (int nt = 0; nt < NT; ++nt) mma_bf16_16816(o[dt][nt], a0, a1, a2, a3, b0[nt], b1[nt]);
+        }
       }
+    }
+    if constexpr (!kEarly) {
+      __syncwarp();
+      if (lane == 0) mbar_arrive(empty_bar);
     }
   }
 
@@ -468,13 +499,14 @@ struct CudaCoreConsumer {
 };
 
 // --------------------------------------------------------------------------
-// One consumer warp's work on one staged block (shared by both schedules).
+// One consumer warp's work on one staged block (shared by both schedules),
+// ending with the stage handed back to the producer.
 // --------------------------------------------------------------------------
 template <int D, int BS, int VAR, int G, int NT>
 __device__ __forceinline__ void consume_block(MmaConsumer<D, BS, NT>& mc,
                                               CudaCoreConsumer<D, BS, (G > 0 ? G : 1)>& cc,
                                               uint32_t sb, float* pbuf, int valid, int pos0,
-                                              float scale_log2, int lane) {
+                                              float scale_log2, int lane, uint32_t empty_bar) {
   using geo = Geo<D, BS>;
   if constexpr (VAR == kMma) {
     if (valid < BS) {
@@ -494,9 +526,11 @@ __device__ __forceinline__ void consume_block(MmaConsumer<D, BS, NT>& mc,
       fence_proxy_async_smem();
       __syncwarp();
     }
-    mc.step(sb, pos0, scale_log2, lane);
+    mc.step(sb, pos0, scale_log2, lane, empty_bar);
   } else {
     cc.step(sb, pbuf, valid, scale_log2, lane);
+    __syncwarp();
+    if (lane == 0) mbar_arrive(empty_bar);
   }
 }
 
@@ -619,9 +653,8 @@ __global__ void __launch_bounds__(kThreads, (VAR == kMma || G <= 2) ? 3 : 2)
       }
       const uint32_t sb = sbase + s * geo::kStageBytes;
       const int valid = (blk0 + i == nblk - 1) ? last_valid : BS;
-      consume_block<D, BS, VAR, G, 1>(mc, cc, sb, pbuf, valid, (blk0 + i) * BS, a.scale_log2, lane);
-      __syncwarp();
-      if (lane == 0) mbar_arrive(bar_empty + 8 * s);
+      consume_block<D, BS, VAR, G, 1>(mc, cc, sb, pbuf, valid, (blk0 + i) * BS, a.scale_log2, lane,
+                                      bar_empty + 8 * s);
     }
   }
   __syncthreads();  // (A) the stage ring is idle; it becomes epilogue scratch
@@ -1023,9 +1056,8 @@ __global__ void __launch_bounds__(kThreads, kStreamCtasPerSm)
           fence_proxy_async_smem();  // the stage goes back to TMA later
           __syncwarp();
         }
-        consume_block<D, BS, VAR, G, NT>(mc, cc, sb, pbuf, valid, blk * BS, a.scale_log2, lane);
-        __syncwarp();
-        if (lane == 0) mbar_arrive(bar_empty + 8 * s);
+        consume_block<D, BS, VAR, G, NT>(mc, cc, sb, pbuf, valid, blk * BS, a.scale_log2, lane,
+                                         bar_empty + 8 * s);
       }
       // ---- segment epilogue: merge the four warps' states
       {
