@@ -1120,8 +1120,8 @@ __global__ void __launch_bounds__(kThreads, kStreamCtasPerSm)
 // CTAs c_first..c_last is merged from their partial slots (slot 0 when the
 // (b, h) is the CTA's first segment, else slot 1).  CTAs with an empty range
 // (more CTAs than units) wrote nothing and are skipped.  Requests of length
-// 0 get zeros here.  Three dependent memory rounds per warp: the prefix
-// sums, every CTA's (m, l) (one per lane), then all partial O rows at once.
+// 0 get zeros here.  Two dependent memory rounds per warp: the prefix sums,
+// then (m, l) and the O row slice of up to 8 covering CTAs at once.
 template <int D, int BS>
 __global__ void __launch_bounds__(128) paged_decode_stream_merge_kernel(const DecodeArgs a,
                                                                         int batch, int ctas) {
@@ -1178,49 +1178,26 @@ __global__ void __launch_bounds__(128) paged_decode_stream_merge_kernel(const De
     if (stream_begin(total, c + 1, ctas) <= cb) return -1;
     return (static_cast<long long>(c) * 2 + (cb >= us ? 0 : 1)) * cols + j;
   };
+  // every lane loads (m, l) and its slice of the O row of up to 8 covering
+  // CTAs at once: a (b, h) split over at most 8 CTAs takes one round of loads
   float mm = -INFINITY, den = 0.f;
-  {
-    float ml[4], ll[4];  // lanes cover up to 128 CTAs per pass
-    for (int c00 = c0; c00 <= c1; c00 += 128) {
-#pragma unroll
-      for (int q = 0; q < 4; ++q) {
-        const int c = c00 + q * 32 + lane;
-        const long long r = c <= c1 ? row_of(c) : -1;
-        ml[q] = r >= 0 ? a.part_m[r] : -INFINITY;
-        ll[q] = r >= 0 ? a.part_l[r] : 0.f;
-      }
-      float m2 = fmaxf(fmaxf(ml[0], ml[1]), fmaxf(ml[2], ml[3]));
-#pragma unroll
-      for (int off = 16; off > 0; off >>= 1) m2 = fmaxf(m2, __shfl_xor_sync(kFull, m2, off));
-      const float mnew = fmaxf(mm, m2);
-      float d2 = 0.f;
-#pragma unroll
-      for (int q = 0; q < 4; ++q)
-        if (ml[q] != -INFINITY) d2 = fmaf(exp2f(ml[q] - mnew), ll[q], d2);
-#pragma unroll
-      for (int off = 16; off > 0; off >>= 1) d2 += __shfl_xor_sync(kFull, d2, off);
-      den = (mm == -INFINITY ? 0.f : den * exp2f(mm - mnew)) + d2;
-      mm = mnew;
-    }
-  }
   float acc[kPer];
 #pragma unroll
   for (int e = 0; e < kPer; ++e) acc[e] = 0.f;
 #pragma unroll 1
   for (int cu = c0; cu <= c1; cu += kUnroll) {
-    float v[kUnroll][kPer];
-    float w[kUnroll];
-    bool ok[kUnroll];
+    float w[kUnroll], lw[kUnroll], v[kUnroll][kPer];
 #pragma unroll
     for (int q = 0; q < kUnroll; ++q) {
       const int c = cu + q;
       const long long r = c <= c1 ? row_of(c) : -1;
-      ok[q] = r >= 0;
-      w[q] = 0.f;
+      w[q] = -INFINITY;
+      lw[q] = 0.f;
 #pragma unroll
       for (int e = 0; e < kPer; ++e) v[q][e] = 0.f;
-      if (ok[q]) {
+      if (r >= 0) {
         w[q] = a.part_m[r];
+        lw[q] = a.part_l[r];
         const float* op = a.part_o + r * D + lane * kPer;
         if constexpr (kPer == 4) {
           const float4 x = *reinterpret_cast<const float4*>(op);
@@ -1235,15 +1212,25 @@ __global__ void __launch_bounds__(128) paged_decode_stream_merge_kernel(const De
         }
       }
     }
+    float mnew = mm;
+#pragma unroll
+    for (int q = 0; q < kUnroll; ++q) mnew = fmaxf(mnew, w[q]);
+    if (mnew == -INFINITY) continue;  // no position seen yet by this column
+    const float f = (mm == -INFINITY) ? 0.f : exp2f(mm - mnew);
+    den *= f;
+#pragma unroll
+    for (int e = 0; e < kPer; ++e) acc[e] *= f;
 #pragma unroll
     for (int q = 0; q < kUnroll; ++q) {
       // a partial whose column saw no position has m = -inf and O = 0
-      if (ok[q] && w[q] != -INFINITY) {
-        const float wq = exp2f(w[q] - mm);
+      if (w[q] != -INFINITY) {
+        const float wq = exp2f(w[q] - mnew);
+        den = fmaf(wq, lw[q], den);
 #pragma unroll
         for (int e = 0; e < kPer; ++e) acc[e] = fmaf(wq, v[q][e], acc[e]);
       }
     }
+    mm = mnew;
   }
   const float inv = den > 0.f ? 1.f / den : 0.f;  // a token that sees nothing gets 0
 #pragma unroll
