@@ -146,6 +146,19 @@ def decode_bytes(lens, hq, hkv, d, bs):
     return kv + qo + tables, kv
 
 
+def workload_config(name, steps_total, world):
+    """The workload fields of the JSON line's ``config``, shared by both arms."""
+    p = workloads.plan(name, extra_tokens=steps_total + 1)
+    s = p.shape
+    batch = len(p.seq_lens) * (p.beams or 1)
+    return {
+        "workload": f"{name}: B{batch} Hq{s.num_q_heads}/Hkv{s.num_kv_heads} D{s.head_dim} bs{s.block_size}",
+        "batch": batch, "num_q_heads": s.num_q_heads, "num_kv_heads": s.num_kv_heads, "head_dim": s.head_dim,
+        "block_size": s.block_size, "num_blocks": p.num_blocks,
+        "parallelism": f"dp{world} (independent batches, no collective)",
+    }
+
+
 def build_cache(name, steps_total, rank, device, prefill=True, variant=0, partition_tokens=0):
     """Pool (seeded bf16 N(0,1)), allocator state and request ids of a workload.
 
@@ -354,15 +367,12 @@ def run_gpu(args):
             "dtype": "bf16",
             "data": "synthetic (seeded bf16 N(0,1) q/K/V; seeded lengths and shuffled block pool)",
             "config": {
-                "workload": f"{args.workload}: B{batch} Hq{cache.hq}/Hkv{cache.hkv} D{cache.d} bs{cache.bs}",
-                "batch": batch, "num_q_heads": cache.hq, "num_kv_heads": cache.hkv, "head_dim": cache.d,
-                "block_size": cache.bs, "num_blocks": cache.num_blocks,
+                **workload_config(args.workload, 2 * (W + K) + 4, world),
                 "mean_seq_len": round(float(np.mean(plans[W][3])), 1),
                 "decode_schedule": (f"balanced persistent: {cache.num_partitions} CTAs"
                                     if cache.schedule == "balanced" else
                                     f"per-partition grid: {cache.num_partitions} partitions"),
                 "l2": f"inputs larger than L2: KV read per step {step_bytes[W][1] / 1e6:.0f} MB > 126 MB",
-                "parallelism": f"dp{world} (independent batches, no collective)",
                 "variant": args.variant,
             },
             "decode_seqs_per_s": round(batch * world * K / (dev_ms * 1e-3), 1),
@@ -494,7 +504,8 @@ def run_reference(args):
         "vs_baseline": None,
         "dtype": "f64",
         "data": "synthetic (seeded bf16 N(0,1) K/V and q, upcast to f64)",
-        "config": {"workload": args.workload,
+        "config": {**workload_config(args.workload, 2 * (args.warmup + args.steps) + 4,
+                                     int(os.environ.get("WORLD_SIZE", "1"))),
                    "note": "each step decodes at least one whole request of the workload on the host"},
         "cpu_baseline": {"value": round(value, 4), "unit": "GB/s", "cores": 1, "kind": "oracle",
                          "sample": runner.describe(n)},
