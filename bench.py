@@ -303,8 +303,8 @@ def run_gpu(args):
 
     # ---- end-to-end arm: per step the host allocator writes the step's
     # metadata into a pinned staging buffer that already holds the step's
-    # q/k/v, one H2D copy moves it all, the device part (fused cache write +
-    # decode + merge) is a CUDA graph replay, and the output comes back
+    # q/k/v; one CUDA graph then copies it to the device, runs the fused
+    # cache write + decode + merge and copies the output back
     for j in range(INPUT_SETS):
         cache.staged("q", j).copy_(qs[j].cpu())
         cache.staged("k", j).copy_(ks[j].cpu())
@@ -317,16 +317,15 @@ def run_gpu(args):
         # step i's metadata was staged in buffer j during step i-1; the
         # allocator work for step i+1 runs while the GPU works on step i
         j = i % INPUT_SETS
-        cache.upload(j)
-        cache.replay(pending.pop(i))
-        h_out.copy_(out, non_blocking=True)
+        cache.replay_step(j, pending.pop(i))  # upload, decode, output copy: one graph
         pending[i + 1] = cache.host_step(ids, (i + 1) % INPUT_SETS)
         stream.synchronize()  # the step's result is on the host
         e2e_lens.append(cache.staged("lens", j).numpy().copy())
 
-    cache.host_step(ids, 0)  # one eager step, then record the graph on its staged data
+    cache.host_step(ids, 0)  # one eager step, then record the graphs on its staged data
     cache.upload(0)
     cache.capture(out)
+    cache.capture_steps(out, h_out)
     pending[0] = cache.host_step(ids, 0)
     for i in range(W):
         e2e_step(i)
@@ -393,10 +392,10 @@ def run_gpu(args):
                 "value": round(e2e_bytes_all / (e2e_ms * 1e-3) / 1e9, 2),
                 "unit": "GB/s",
                 "h2d_bytes_per_step": int(e2e_h2d / K),
-                "path": "per step: one H2D copy of a pinned staging buffer (metadata from the C++ "
-                        "allocator + the step's q/k/v), CUDA-graph replay of fused cache write + decode "
-                        "+ merge, D2H of the output, sync; the allocator work for the next step runs "
-                        "on the host while the GPU works",
+                "path": "per step: one CUDA graph holding the H2D copy of a pinned staging buffer "
+                        "(metadata from the C++ allocator + the step's q/k/v), the fused cache write + "
+                        "decode + merge and the D2H copy of the output; then a sync; the allocator work "
+                        "for the next step runs on the host while the GPU works",
                 "d2h_bytes_per_step": int(h_out.nbytes),
                 "ms_per_step": round(e2e_ms / K, 5),
             },

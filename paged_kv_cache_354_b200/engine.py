@@ -151,6 +151,35 @@ class PagedDecodeCache:
             pa_copy_blocks(self.pool, self.s_pairs[:npairs])
         self.graph.replay()
 
+    def capture_steps(self, out, h_out):
+        """Record, for every staging buffer j, a whole step as one CUDA graph:
+        the upload of buffer j, the fused cache write + decode + merge, and the
+        copy of ``out`` into the pinned host tensor ``h_out``.  Needs the graph
+        of ``capture`` (used for steps with copy-on-write pairs, whose copies
+        must run between the upload and the decode)."""
+        assert self.graph is not None, "capture() first"
+        self._out, self._h_out = out, h_out
+        self.step_graphs = []
+        for j in range(len(self.h_stage)):
+            g = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(g):
+                self.d_stage.copy_(self.h_stage[j], non_blocking=True)
+                self._device_step(out)
+                h_out.copy_(out, non_blocking=True)
+            self.step_graphs.append(g)
+
+    def replay_step(self, j, npairs):
+        """A whole staged step (asynchronous): one graph launch, or, with
+        copy-on-write pairs, the upload, the copies, the decode graph and the
+        output copy in turn.  ``h_out`` holds the output once the stream is
+        synchronised."""
+        if npairs:
+            self.upload(j)
+            self.replay(npairs)
+            self._h_out.copy_(self._out, non_blocking=True)
+        else:
+            self.step_graphs[j].replay()
+
     # -------------------------------------------------------------- device
     def run(self, q, k_new, v_new, out, slots, tables, lens, pairs=None, max_seq_len=None):
         """Device part of a step on already-resident inputs (async): the

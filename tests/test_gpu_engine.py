@@ -93,3 +93,75 @@ def test_graph_replayed_steps_match_oracle(schedule):
         compare(out.double().cpu().numpy(), want)
     assert seen_cow == 4  # 2 + 2 beams copy their prompt's shared partial block on step 0
     assert pk.pa_device_error() == 0
+
+
+def test_whole_step_graphs_match_oracle():
+    """capture_steps: upload, fused decode and output copy as one graph per
+    staging buffer (steps with copy-on-write pairs -- here step 3 -- take the
+    eager upload and copies); every step's host output equals the oracle's
+    replay, and the pool equals the oracle's bit for bit."""
+    dev = torch.device("cuda", torch.cuda.current_device())
+    hq, hkv, d, bs, sets = 8, 2, 128, 16, 3
+    nb = 200
+    order = np.random.default_rng(11).permutation(nb)
+    cache = PagedDecodeCache(nb, hq, hkv, d, bs, max_batch=4, max_seq_len=700, initial_order=order,
+                             device=dev, staging_sets=sets)
+    ref = BlockAllocator(nb, bs, order)
+    gen = torch.Generator(device=dev)
+    gen.manual_seed(12)
+    cache.pool.copy_(torch.randn(cache.pool.shape, generator=gen, device=dev).bfloat16())
+    pool_ref = bits(cache.pool)
+    for a in (cache.alloc, ref):
+        a.add_seq(0)
+        a.append(0, 300 + 5)
+        a.fork(0, 1)  # shares a partial block: the first step copies it
+        for sid, n in ((2, 17), (3, 640)):
+            a.add_seq(sid)
+            a.append(sid, n)
+    ids = [0, 1, 2, 3]
+    out = torch.empty((4, hq, d), dtype=torch.bfloat16, device=dev)
+    h_out = torch.empty(out.shape, dtype=out.dtype).pin_memory()
+    scale = 1.0 / math.sqrt(d)
+    inputs = []
+    for step in range(7):
+        g = torch.Generator().manual_seed(50 + step)
+        inputs.append(tuple(torch.randn(shape, generator=g).bfloat16()
+                            for shape in ((4, hq, d), (4, hkv, d), (4, hkv, d))))
+    for j in range(sets):  # the first steps' inputs, as the loop below stages them
+        for name, t in zip("qkv", inputs[j]):
+            cache.staged(name, j).copy_(t)
+    npairs = cache.host_step(ids, 0)
+    assert npairs == 1
+    cache.upload(0)
+    pk.pa_copy_blocks(cache.pool, cache.s_pairs[:npairs])
+    cache.capture(out)  # its warm-up performs step 0
+    cache.capture_steps(out, h_out)
+    torch.cuda.synchronize()
+    seen = 0
+    for step in range(7):
+        j = step % sets
+        if step == 3:  # request 2 restarts as a fork of request 3: its first write copies
+            for a in (cache.alloc, ref):
+                a.free_seq(2)
+                a.fork(3, 2)
+        if step > 0:
+            for name, t in zip("qkv", inputs[step]):
+                cache.staged(name, j).copy_(t)
+            npairs = cache.host_step(ids, j)
+            assert npairs == (1 if step == 3 else 0)
+            cache.replay_step(j, npairs)
+        else:
+            h_out.copy_(out)
+        torch.cuda.synchronize()
+        slots, pairs = ref.append_batch(ids, 1)
+        assert len(pairs) == npairs
+        seen += npairs
+        opa.copy_blocks(pool_ref, pairs)
+        qh, kh, vh = inputs[step]
+        opa.reshape_and_cache(pool_ref, bits(kh), bits(vh), np.array(slots))
+        tables, lens = workloads.block_tables(ref, ids, cache.max_blocks)
+        want = opa.decode(qh.double().numpy(), u16_to_f64(pool_ref), tables, lens, scale)
+        compare(h_out.double().numpy(), want)
+    assert seen == 2
+    assert np.array_equal(bits(cache.pool), pool_ref)
+    assert pk.pa_device_error() == 0
