@@ -135,12 +135,13 @@ struct MmaConsumer {
 
   // qbase: Q row of (token 0, head 0) of this KV head's group; consecutive
   // tokens are q_tok_stride elements apart, heads D apart.
+  // col0: the first of the warp's 8 * NT columns (a warp pair splits 16).
   __device__ __forceinline__ void init(const __nv_bfloat16* qbase, int cols, int group, int qtok,
-                                       size_t q_tok_stride, int len, int lane) {
+                                       size_t q_tok_stride, int len, int lane, int col0 = 0) {
     const int c = 2 * (lane & 3);
 #pragma unroll
     for (int nt = 0; nt < NT; ++nt) {
-      const int col = nt * 8 + (lane >> 2);  // B-operand column of this thread
+      const int col = col0 + nt * 8 + (lane >> 2);  // B-operand column of this thread
       const bool real = col < cols;
       const int t = real ? col / group : 0;
       const __nv_bfloat16* qr = qbase + t * q_tok_stride + (col - t * group) * D + c;
@@ -151,7 +152,7 @@ struct MmaConsumer {
       }
 #pragma unroll
       for (int e = 0; e < 2; ++e) {
-        const int cc = nt * 8 + c + e;  // accumulator column of this thread
+        const int cc = col0 + nt * 8 + c + e;  // accumulator column of this thread
         lim[nt][e] = cc < cols ? len - qtok + cc / group : len - 1;
         m[nt][e] = -INFINITY;
         l[nt][e] = 0.f;
@@ -749,19 +750,30 @@ __global__ void __launch_bounds__(kThreads, (VAR == kMma || G <= 2) ? 3 : 2)
 constexpr int kStreamCtasPerSm = PA_STREAM_CTAS_PER_SM;
 constexpr int kStreamMaxBatch = 4096;  // the prefix table lives in shared memory
 
+// Consumer groups of the balanced kernel: with up to 8 (token, head) columns
+// each consumer warp takes every fourth block alone; with 16 (two 8-wide MMA
+// tiles) the warps pair up, both warps of a pair take every other block and
+// each computes 8 of the columns, so no warp carries the 16-column tile's
+// registers and every pair keeps twice as many stages in flight.
+template <int NT>
+struct StreamGroups {
+  static constexpr int kPerGroup = NT == 2 ? 2 : 1;          // warps sharing a block
+  static constexpr int kGroups = kConsumerWarps / kPerGroup;  // block streams per CTA
+};
+
 template <int D, int BS, int G, int NT>
 struct StreamSmem {
   using geo = Geo<D, BS>;
-  static constexpr int kCols = 8 * NT;  // epilogue rows per warp: (token, head) columns
-  // Stage s must always be consumed by warp s % kConsumerWarps: a warp then
-  // takes a stage's rounds one after the other, so a parity wait (which
-  // only tells the current phase from the previous one) never runs two
-  // rounds ahead.  Hence a whole multiple of the consumer warp count.
-  static constexpr int kRingStages =
-      (PA_STREAM_RING_BYTES / geo::kStageBytes) / kConsumerWarps * kConsumerWarps;
-  static constexpr int kStages = kRingStages > kConsumerWarps ? kRingStages : kConsumerWarps;
-  static_assert(kStages >= kConsumerWarps && kStages % kConsumerWarps == 0,
-                "stages must be a positive multiple of the consumer warps");
+  static constexpr int kCols = 8;  // epilogue rows per warp: its (token, head) columns
+  // Stage s must always be consumed by group s % kGroups: a group then takes
+  // a stage's rounds one after the other, so a parity wait (which only tells
+  // the current phase from the previous one) never runs two rounds ahead.
+  // Hence a whole multiple of the consumer group count.
+  static constexpr int kGroups = StreamGroups<NT>::kGroups;
+  static constexpr int kRingStages = (PA_STREAM_RING_BYTES / geo::kStageBytes) / kGroups * kGroups;
+  static constexpr int kStages = kRingStages > kGroups ? kRingStages : kGroups;
+  static_assert(kStages >= kGroups && kStages % kGroups == 0,
+                "stages must be a positive multiple of the consumer groups");
   static constexpr int kBar = kStages * geo::kStageBytes;         // full[S], empty[S]
   static constexpr int kMisc = kBar + 16 * kStages;               // last_round[S], abort
   static constexpr int kScan = (kMisc + 4 * kStages + 4 + 15) & ~15;  // scan scratch
@@ -890,6 +902,7 @@ __global__ void __launch_bounds__(kThreads, kStreamCtasPerSm)
                                int batch) {
   using geo = Geo<D, BS>;
   using sm = StreamSmem<D, BS, G, NT>;
+  using grp = StreamGroups<NT>;
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw_base = smem_u32(smem_raw);
   const uint32_t pad = ((raw_base + 1023u) & ~1023u) - raw_base;
@@ -909,7 +922,7 @@ __global__ void __launch_bounds__(kThreads, kStreamCtasPerSm)
   if (threadIdx.x == 0) {  // shared memory only: may overlap the previous grid
     for (int s = 0; s < sm::kStages; ++s) {
       mbar_init(bar_full + 8 * s, 1);
-      mbar_init(bar_empty + 8 * s, 1);
+      mbar_init(bar_empty + 8 * s, grp::kPerGroup);
       last_round[s] = -1;
     }
     *abort_flag = 0;
@@ -926,7 +939,7 @@ __global__ void __launch_bounds__(kThreads, kStreamCtasPerSm)
   const long long u_end = stream_begin(total, blockIdx.x + 1, ctas);
   if (u_begin >= u_end) return;  // uniform: this CTA has no units
 
-  [[maybe_unused]] MmaConsumer<D, BS, NT> mc;
+  [[maybe_unused]] MmaConsumer<D, BS, 1> mc;  // one 8-column tile per warp
   [[maybe_unused]] CudaCoreConsumer<D, BS, (G > 0 ? G : 1)> cc;
   if (warp == kConsumerWarps) {
     // ------------------------------------------------------------ producer
@@ -996,6 +1009,8 @@ __global__ void __launch_bounds__(kThreads, kStreamCtasPerSm)
     float* l_all = m_all + kConsumerWarps * kC;
     const int cols = a.cols;
     const size_t q_tok_stride = static_cast<size_t>(a.num_q_heads) * D;
+    const int grp_id = warp / grp::kPerGroup;  // block stream of this warp
+    const int sub = warp % grp::kPerGroup;     // its 8 columns within the group's 16
     int b, h, k;
     stream_locate(prefix, batch, hkv, u_begin, b, h, k);
     long long u = u_begin;
@@ -1010,14 +1025,15 @@ __global__ void __launch_bounds__(kThreads, kStreamCtasPerSm)
       const int len = effective_len(__ldg(a.seq_lens + b), BS, a, false);
       const int last_valid = len - (nb - 1) * BS;
       const __nv_bfloat16* qbase = a.q + qrow0 * D;
-      if constexpr (VAR == kMma) mc.init(qbase, cols, g, a.qtok, q_tok_stride, len, lane);
+      if constexpr (VAR == kMma) mc.init(qbase, cols, g, a.qtok, q_tok_stride, len, lane, 8 * sub);
       else cc.init(qbase, lane);
       // fused cache write: the warp that takes this (b, h)'s last block
       // fetches the new K/V row now and patches it into the staged tile
       const int last_ii = i + cnt - 1;
       bool patch = false;
       uint4 new_row = make_uint4(0u, 0u, 0u, 0u);
-      if (a.new_k != nullptr && k + cnt == nb && last_ii % kConsumerWarps == warp) {
+      // (never with warp pairs: several query tokens, and no cache write)
+      if (grp::kPerGroup == 1 && a.new_k != nullptr && k + cnt == nb && last_ii % kConsumerWarps == warp) {
         patch = __ldg(a.new_slots + b) >= 0;
         if (patch && lane < 2 * (D / 8)) {
           const uint4* src = (lane < D / 8 ? a.new_k : a.new_v) +
@@ -1026,9 +1042,9 @@ __global__ void __launch_bounds__(kThreads, kStreamCtasPerSm)
         }
       }
       // this warp's blocks of the segment: running indices i..i+cnt-1 that are
-      // congruent to the warp number
-      for (int ii = i + ((warp - i % kConsumerWarps + kConsumerWarps) % kConsumerWarps);
-           ii < i + cnt; ii += kConsumerWarps) {
+      // congruent to its group number
+      for (int ii = i + ((grp_id - i % grp::kGroups + grp::kGroups) % grp::kGroups); ii < i + cnt;
+           ii += grp::kGroups) {
         if (*abort_flag) break;
         const int s = ii % sm::kStages;
         if (!mbar_wait(bar_full + 8 * s, (ii / sm::kStages) & 1)) {
@@ -1056,10 +1072,11 @@ __global__ void __launch_bounds__(kThreads, kStreamCtasPerSm)
           fence_proxy_async_smem();  // the stage goes back to TMA later
           __syncwarp();
         }
-        consume_block<D, BS, VAR, G, NT>(mc, cc, sb, pbuf, valid, blk * BS, a.scale_log2, lane,
-                                         bar_empty + 8 * s);
+        consume_block<D, BS, VAR, G, 1>(mc, cc, sb, pbuf, valid, blk * BS, a.scale_log2, lane,
+                                        bar_empty + 8 * s);
       }
-      // ---- segment epilogue: merge the four warps' states
+      // ---- segment epilogue: merge the warps' states (column c lives in the
+      // scratch rows of the group members that computed it)
       {
         float* o_s = o_all + warp * kC * geo::kOStride;
         if constexpr (VAR == kMma) mc.store(o_s, m_all + warp * kC, l_all + warp * kC, kC, lane);
@@ -1072,16 +1089,20 @@ __global__ void __launch_bounds__(kThreads, kStreamCtasPerSm)
         for (int idx = threadIdx.x; idx < cols * D / 2; idx += kConsumerWarps * 32) {
           const int c = (2 * idx) / D;  // column: token c / g, head c % g
           const int d = (2 * idx) % D;
+          const int csub = grp::kPerGroup == 2 ? (c >> 3) : 0;  // which member of a group
+          const int cr = c - 8 * csub;                           // row in that member's scratch
           float mm = -INFINITY;
 #pragma unroll
-          for (int w = 0; w < kConsumerWarps; ++w) mm = fmaxf(mm, m_all[w * kC + c]);
+          for (int gi = 0; gi < grp::kGroups; ++gi)
+            mm = fmaxf(mm, m_all[(gi * grp::kPerGroup + csub) * kC + cr]);
           float ll = 0.f, v0 = 0.f, v1 = 0.f;
 #pragma unroll
-          for (int w = 0; w < kConsumerWarps; ++w) {
-            const float mw = m_all[w * kC + c];
+          for (int gi = 0; gi < grp::kGroups; ++gi) {
+            const int w = gi * grp::kPerGroup + csub;
+            const float mw = m_all[w * kC + cr];
             const float f = (mw == -INFINITY) ? 0.f : exp2f(mw - mm);
-            const float* ow = o_all + (w * kC + c) * geo::kOStride + d;
-            ll = fmaf(f, l_all[w * kC + c], ll);
+            const float* ow = o_all + (w * kC + cr) * geo::kOStride + d;
+            ll = fmaf(f, l_all[w * kC + cr], ll);
             v0 = fmaf(f, ow[0], v0);
             v1 = fmaf(f, ow[1], v1);
           }
