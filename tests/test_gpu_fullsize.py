@@ -90,3 +90,44 @@ def test_full_size_sampled(name):
         errs.append(np.abs(got[b, j] - want))
     errs = np.concatenate(errs)
     assert errs.max() <= MAX_ABS and errs.mean() <= MEAN_ABS, (errs.max(), errs.mean())
+
+
+def test_full_size_multi_token_sampled():
+    """pa_decode_multi at the Llama-3-8B decode shape with 4 causal query
+    tokens per request (16 columns per KV head: the paired-warp kernel), the
+    configuration of bench.py's multi-token study; sampled (request, token,
+    head) outputs against the oracle over each token's visible prefix."""
+    dev = torch.device("cuda", torch.cuda.current_device())
+    p, cache, ids, gen = bench.build_cache("llama8b", 2, 0, dev, prefill=False)
+    s = p.shape
+    T = 4
+    pool_u16 = bits(cache.pool)
+    tables, lens = cache.alloc.block_tables(ids, cache.max_blocks)
+    q = torch.randn((len(ids), T, s.num_q_heads, s.head_dim), generator=gen, device=dev).bfloat16()
+    out = torch.full_like(q, float("nan"))
+    scale = 1.0 / math.sqrt(s.head_dim)
+    ws = torch.empty(max(256, pk.pa_decode_multi_workspace_size(len(ids), T, s.num_q_heads, s.num_kv_heads,
+                                                                 s.head_dim, s.block_size, cache.max_seq_len)),
+                     dtype=torch.uint8, device=dev)
+    pk.pa_device_error(clear=True)
+    pk.pa_decode_multi(out, q, cache.pool, torch.as_tensor(tables, device=dev), torch.as_tensor(lens, device=dev),
+                       cache.max_seq_len, scale, ws)
+    torch.cuda.synchronize()
+    assert pk.pa_device_error() == 0
+    assert torch.isfinite(out).all()
+    q64 = q.double().cpu().numpy()
+    got = out.double().cpu().numpy()
+    rng = np.random.default_rng(4242)
+    g = s.num_q_heads // s.num_kv_heads
+    errs = []
+    for b in [int(x) for x in rng.integers(0, len(ids), SAMPLES)]:
+        t = int(rng.integers(0, T))
+        j = int(rng.integers(0, s.num_q_heads))
+        h = j // g
+        visible = int(lens[b]) - T + t + 1
+        nblk = -(-visible // s.block_size)
+        mini = u16_to_f64(pool_u16[tables[b, :nblk]][:, :, h:h + 1])
+        want = opa.decode_one(q64[b, t, j], mini, np.arange(nblk), visible, 0, scale)
+        errs.append(np.abs(got[b, t, j] - want))
+    errs = np.concatenate(errs)
+    assert errs.max() <= MAX_ABS and errs.mean() <= MEAN_ABS, (errs.max(), errs.mean())
