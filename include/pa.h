@@ -178,7 +178,7 @@ int pa_decode(pa_bf16* out, const pa_bf16* q, const pa_bf16* kv_pool,
 
 /* Kernel variant of the decode main loop. */
 typedef enum pa_decode_variant {
-  PA_DECODE_AUTO = 0,      /* tensor cores (mma) for group >= 4, else CUDA cores */
+  PA_DECODE_AUTO = 0,      /* tensor cores (mma) for every group: faster at every size measured */
   PA_DECODE_CUDA_CORE = 1, /* fp32 FMA on CUDA cores (group 1, 2 or 4) */
   PA_DECODE_MMA = 2        /* bf16 mma.sync with fp32 accumulate (group 1..8) */
 } pa_decode_variant;

@@ -16,12 +16,12 @@
 //  * four consumer warps each own every fourth block and keep their own
 //    online-softmax state; the query heads of a GQA group share every loaded
 //    tile;
-//  * consumer math: for groups >= 4 (and on request) bf16 mma.sync with
+//  * consumer math: by default bf16 mma.sync with
 //    fp32 accumulate in a transposed form, S^T = K Q^T then O^T += V^T P^T,
 //    so the 16-row side of the MMA is the token / head-dim axis and the
 //    group of g <= 8 query heads fills the 8-wide side; P^T is formed from
-//    the S^T accumulators in registers with movmatrix.  For groups <= 2,
-//    fp32 FMA on CUDA cores;
+//    the S^T accumulators in registers with movmatrix.  On request, for
+//    groups 1, 2 and 4, fp32 FMA on CUDA cores;
 //  * the warps' partial states merge through shared memory; a sequence cut
 //    into several partitions writes fp32 partials (O, running max, sum) and
 //    a second kernel merges them with the log-sum-exp rule.
@@ -1522,7 +1522,9 @@ static int decode_impl(pa_bf16* out, const pa_bf16* q, const pa_bf16* kv_pool,
                 2 * kMaxGroup);
   if (qtok > 1 && variant == kCudaCore)
     return fail(PA_ERR_UNSUPPORTED, "multi-token decode has the tensor-core variant only");
-  if (variant == PA_DECODE_AUTO) variant = (group >= 4 || qtok > 1) ? kMma : kCudaCore;
+  // tensor cores for every group: at scale they beat the CUDA-core consumer
+  // even where the group leaves most of the 8-wide tile empty (g = 1, 2)
+  if (variant == PA_DECODE_AUTO) variant = kMma;
   if (variant == kCudaCore && group != 1 && group != 2 && group != 4)
     return fail(PA_ERR_UNSUPPORTED, "pa_decode: CUDA-core variant has no group size %d", group);
   if (variant != kCudaCore && variant != kMma)
@@ -1638,7 +1640,7 @@ static int decode_contiguous_impl(pa_bf16* out, const pa_bf16* q, const pa_bf16*
   if (!a16(out) || !a16(q) || !a16(kv_cache) || (reinterpret_cast<uintptr_t>(seq_lens) & 3u))
     return fail(PA_ERR_INVALID, "pa_decode_contiguous: misaligned pointer");
   const int group = hq / hkv;
-  if (variant == PA_DECODE_AUTO) variant = group >= 4 ? kMma : kCudaCore;
+  if (variant == PA_DECODE_AUTO) variant = kMma;
   if (variant != kCudaCore && variant != kMma)
     return fail(PA_ERR_INVALID, "pa_decode_contiguous: unknown variant %d", variant);
   if (variant == kCudaCore && group != 1 && group != 2 && group != 4)
