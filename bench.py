@@ -687,6 +687,58 @@ def study_multi_token(iters=30):
     assert pk.pa_device_error() == 0
 
 
+def study_variants(iters=20):
+    """Tensor-core vs CUDA-core consumer across GQA group sizes: pa_decode on
+    the llama8b lengths and shuffled pool, Hkv in {8, 32}, head dim 128 and
+    (Hkv 8) 64, groups 1, 2, 4, 8; CUDA events over back-to-back launches."""
+    import torch
+
+    import paged_kv_cache_354_b200 as pk
+
+    dev = torch.device("cuda", torch.cuda.current_device())
+    p = workloads.plan("llama8b")
+    gen = torch.Generator(device=dev)
+    gen.manual_seed(workloads.seed_of("llama8b"))
+    ws = torch.empty(64 << 20, dtype=torch.uint8, device=dev)
+    for hkv, d in ((8, 128), (32, 128), (8, 64)):
+        bs = 16
+        pool = torch.randn((p.num_blocks, 2, hkv, bs, d), generator=gen, device=dev).bfloat16()
+        alloc = pk.PaAlloc(p.num_blocks, bs, p.initial_order)
+        ids = workloads.populate(alloc, p)
+        tables, lens = alloc.block_tables(ids, -(-int(max(p.seq_lens)) // bs))
+        d_t, d_l = torch.as_tensor(tables, device=dev), torch.as_tensor(lens, device=dev)
+        for g in (1, 2, 4, 8):
+            q = torch.randn((len(ids), hkv * g, d), generator=gen, device=dev).bfloat16()
+            out = torch.empty_like(q)
+            nbytes = decode_bytes(lens, hkv * g, hkv, d, bs)[0]
+            res = {}
+            for name, variant in (("mma", pk.PA_DECODE_MMA), ("cuda_core", pk.PA_DECODE_CUDA_CORE)):
+                if variant == pk.PA_DECODE_CUDA_CORE and g not in (1, 2, 4):
+                    continue
+
+                def call():
+                    pk.pa_decode(out, q, pool, d_t, d_l, int(lens.max()), 1.0 / math.sqrt(d), workspace=ws,
+                                 variant=variant)
+
+                for _ in range(3):
+                    call()
+                torch.cuda.synchronize()
+                e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+                e0.record()
+                for _ in range(iters):
+                    call()
+                e1.record()
+                torch.cuda.synchronize()
+                res[name] = e0.elapsed_time(e1) / iters * 1e3
+            print(json.dumps({"study": "variants", "workload": "llama8b lengths", "num_kv_heads": hkv,
+                              "head_dim": d, "group": g, **{f"{k}_us": round(v, 1) for k, v in res.items()},
+                              **{f"{k}_gbs": round(nbytes / v / 1e3, 1) for k, v in res.items()},
+                              "iters": iters}), flush=True)
+        del pool
+        torch.cuda.empty_cache()
+    assert pk.pa_device_error() == 0
+
+
 def study_read_bandwidth(iters=20):
     """What a plain contiguous read stream reaches on this GPU: torch's own
     bf16 sum (fp32 accumulate) over 2 GiB, for context beside the copy-based
@@ -718,7 +770,7 @@ def main():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--variant", default="auto", choices=["auto", "mma", "cuda_core"],
                     help="decode consumer: auto (tensor cores for GQA groups >= 4), or forced")
-    ap.add_argument("--study", choices=["memory-waste", "page-table", "multi-token", "read-bandwidth"],
+    ap.add_argument("--study", choices=["memory-waste", "page-table", "multi-token", "read-bandwidth", "variants"],
                     help="print the study's JSON lines instead of the benchmark line")
     ap.add_argument("--partition-tokens", type=int, default=0,
                     help="0 = library's choice; -1 = balanced schedule; N > 0 = per-partition grid of "
@@ -736,6 +788,8 @@ def main():
         study_multi_token()
     elif args.study == "read-bandwidth":
         study_read_bandwidth()
+    elif args.study == "variants":
+        study_variants()
     elif args.impl == "reference":
         run_reference(args)
     else:
