@@ -39,6 +39,7 @@ import workloads  # noqa: E402
 METRIC = "paged-decode KV-read GB/s & % of HBM peak; decode seqs/s at Llama-3-8B shape"
 PEAKS_FALLBACK = {"hbm_gbs": 6650.0, "source": "fallback"}
 INPUT_SETS = 4  # distinct q/k/v sets cycled through the steps
+SPEC_HBM_GBS = 8000.0  # B200 data-sheet HBM3e bandwidth
 
 
 TRAFFIC_FILE = os.path.join(ROOT, "profiles", "paged_decode_traffic.json")
@@ -376,6 +377,9 @@ def run_gpu(args):
             },
             "decode_seqs_per_s": round(batch * world * K / (dev_ms * 1e-3), 1),
             "frac_of_hbm_peak": round(gbs / world / peaks["hbm_gbs"], 4),
+            # against the B200 data-sheet bandwidth (8 TB/s) rather than the measured copy
+            "frac_of_spec_hbm": round(gbs / world / SPEC_HBM_GBS, 4),
+            "spec_hbm_gbs": SPEC_HBM_GBS,
             "roofline": {
                 "bound": "hbm",
                 "kernel": "pa_decode (main + split-K merge), K back-to-back launches",
