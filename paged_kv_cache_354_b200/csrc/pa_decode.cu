@@ -87,6 +87,7 @@ struct DecodeArgs {
   int32_t* err;
   int num_q_heads, num_kv_heads, group;
   int num_blocks, max_blocks_per_seq;
+  int len_cap;  // > 0: the longest length the table row holds (else max_blocks_per_seq * bs)
   int part_blocks, max_parts;
   float scale_log2;  // scale * log2(e)
   int* stream_prefix;  // balanced schedule: per-request block-count prefix sums [B+1]
@@ -105,7 +106,7 @@ struct DecodeArgs {
 // (both kernels use this, so they agree on the partition count).
 __device__ __forceinline__ int effective_len(int raw, int bs, const DecodeArgs& a, bool report) {
   int len = raw < 0 ? 0 : raw;
-  const int cap_table = a.max_blocks_per_seq * bs;
+  const int cap_table = a.len_cap > 0 ? a.len_cap : a.max_blocks_per_seq * bs;
   const long long cap_grid = static_cast<long long>(a.max_parts) * a.part_blocks * bs;
   if (len > cap_table || len > cap_grid || raw < 0) {
     if (report) flag_error(a.err, PA_DEVERR_SEQ_LEN);
@@ -894,7 +895,10 @@ __device__ __forceinline__ void consumer_bar() {
 // [NB][2][Hkv][bs][D] through the block table.  kContiguous: one reserved
 // run per request, [B][2][Hkv][max_len][D], block k being rows
 // [k bs, (k+1) bs) -- no table; the naive layout paging replaces.
-enum Layout { kPaged = 0, kContiguous = 1 };
+// kPagedPairs: the pool of 16-token blocks with head dim 64, taken two
+// table entries per 32-token tile (each block's 2 KiB K and V planes
+// would otherwise make stages too small for the per-stage costs).
+enum Layout { kPaged = 0, kContiguous = 1, kPagedPairs = 2 };
 
 template <int D, int BS, int VAR, int G, int NT, int LAYOUT = kPaged>
 __global__ void __launch_bounds__(kThreads, kStreamCtasPerSm)
@@ -952,21 +956,32 @@ __global__ void __launch_bounds__(kThreads, kStreamCtasPerSm)
     while (u < u_end && !stop) {
       const int nb = prefix[b + 1] - prefix[b];
       const int cnt = static_cast<int>(min(static_cast<long long>(nb - k), u_end - u));
-      for (int base = 0; base < cnt && !stop; base += 32) {
+      constexpr int kPerFetch = LAYOUT == kPagedPairs ? 16 : 32;  // tiles per table fetch
+      // physical blocks of request b (the pair layout's last tile may hold one)
+      const int nphys = LAYOUT == kPagedPairs
+                            ? (effective_len(__ldg(a.seq_lens + b), BS, a, false) + BS / 2 - 1) / (BS / 2)
+                            : 0;
+      for (int base = 0; base < cnt && !stop; base += kPerFetch) {
         int phys = 0;
-        if constexpr (LAYOUT == kPaged) {
-          const int32_t* trow = a.block_tables + static_cast<size_t>(b) * a.max_blocks_per_seq + k;
-          if (base + lane < cnt) {
-            phys = __ldg(trow + base + lane);
+        if constexpr (LAYOUT == kPaged || LAYOUT == kPagedPairs) {
+          const int32_t* trow = a.block_tables + static_cast<size_t>(b) * a.max_blocks_per_seq;
+          // kPaged: entry k + base + lane; pairs: entry 2 (k + base) + lane
+          const int e = LAYOUT == kPaged ? k + base + lane : 2 * (k + base) + lane;
+          const bool in = LAYOUT == kPaged ? base + lane < cnt : (e < 2 * (k + cnt) && e < nphys);
+          phys = -1;
+          if (in) {
+            phys = __ldg(trow + e);
             if (static_cast<unsigned>(phys) >= static_cast<unsigned>(a.num_blocks)) {
               flag_error(a.err, PA_DEVERR_BLOCK_ID);
               phys = 0;  // read a valid block instead; the result is flagged as wrong
             }
           }
         }
-        const int n32 = min(32, cnt - base);
+        const int n32 = min(kPerFetch, cnt - base);
         for (int j = 0; j < n32; ++j) {
-          const int pb = (LAYOUT == kPaged) ? __shfl_sync(kFull, phys, j) : 0;
+          const int pb = (LAYOUT == kPaged) ? __shfl_sync(kFull, phys, j)
+                                            : (LAYOUT == kPagedPairs ? __shfl_sync(kFull, phys, 2 * j) : 0);
+          const int pb1 = (LAYOUT == kPagedPairs) ? __shfl_sync(kFull, phys, 2 * j + 1) : -1;
           int failed = 0;
           if (lane == 0) {
             const int ii = i + base + j;
@@ -978,13 +993,27 @@ __global__ void __launch_bounds__(kThreads, kStreamCtasPerSm)
               failed = 1;
             } else {
               const uint32_t fb = bar_full + 8 * s;
-              mbar_arrive_expect_tx(fb, geo::kStageBytes);
               const uint32_t dst = sbase + s * geo::kStageBytes;
+              if constexpr (LAYOUT == kPagedPairs) {
+                // K then V rows of the tile's first block, the second block's
+                // below them (16 rows = 2 KiB each); a missing second block
+                // leaves rows 16..31 stale, which the consumer masks
+                static_assert(D == 64 && BS == 32, "pairs of 16-token blocks, head dim 64");
+                mbar_arrive_expect_tx(fb, pb1 >= 0 ? geo::kStageBytes : geo::kStageBytes / 2);
+                tma_load_3d(dst, &kv_map, fb, 0, h * (BS / 2), 2 * pb);
+                tma_load_3d(dst + BS * 128, &kv_map, fb, 0, h * (BS / 2), 2 * pb + 1);
+                if (pb1 >= 0) {
+                  tma_load_3d(dst + (BS / 2) * 128, &kv_map, fb, 0, h * (BS / 2), 2 * pb1);
+                  tma_load_3d(dst + (BS + BS / 2) * 128, &kv_map, fb, 0, h * (BS / 2), 2 * pb1 + 1);
+                }
+              } else {
+                mbar_arrive_expect_tx(fb, geo::kStageBytes);
+              }
               if constexpr (LAYOUT == kPaged) {
 #pragma unroll
                 for (int x = 0; x < geo::kRegions; ++x)
                   tma_load_3d(dst + x * geo::kRegionBytes, &kv_map, fb, x * 64, h * BS, 2 * pb);
-              } else {  // rows of block k + base + j of request b, head h; keys then values
+              } else if constexpr (LAYOUT == kContiguous) {  // rows of block k + base + j of request b
 #pragma unroll
                 for (int x = 0; x < geo::kRegions; ++x)
                   tma_load_4d(dst + x * geo::kRegionBytes, &kv_map, fb, x * 64, (k + base + j) * BS, h, 2 * b);
@@ -1354,6 +1383,10 @@ static size_t align256(size_t x) { return (x + 255) & ~static_cast<size_t>(255);
 // work), kForceBalanced = balanced, > 0 = per-partition grid with
 // partitions of that many tokens.
 constexpr int kForceBalanced = -1;
+// Tokens per tile of the balanced schedule: one block, or two blocks for
+// 16-token blocks of head dim 64 (kPagedPairs).
+static int stream_tile(int d, int bs) { return (d == 64 && bs == 16) ? 2 * bs : bs; }
+
 static int make_plan(int batch, int hq, int hkv, int d, int bs, int max_seq_len,
                      int partition_tokens, Plan* plan, int qtok = 1) {
   const int nblk_max = max_seq_len > 0 ? (max_seq_len + bs - 1) / bs : 1;
@@ -1362,9 +1395,11 @@ static int make_plan(int batch, int hq, int hkv, int d, int bs, int max_seq_len,
     return fail(PA_ERR_UNSUPPORTED, "multi-token decode runs on the balanced schedule only");
   if (qtok > 1) partition_tokens = kForceBalanced;
   const int sms = sm_count() > 0 ? sm_count() : 148;
-  // the balanced schedule pays when there are at least a few blocks per
+  // the balanced schedule pays when there are at least a few tiles per
   // persistent CTA; tiny batches (launch-bound anyway) take the grid
-  const long long units_max = static_cast<long long>(batch) * hkv * nblk_max;
+  const int tile = stream_tile(d, bs);
+  const long long units_max =
+      static_cast<long long>(batch) * hkv * (max_seq_len > 0 ? (max_seq_len + tile - 1) / tile : 1);
   if (partition_tokens == kForceBalanced && batch > kStreamMaxBatch)
     return fail(PA_ERR_UNSUPPORTED, "balanced schedule: batch %d above %d", batch, kStreamMaxBatch);
   if (partition_tokens == kForceBalanced ||
@@ -1487,6 +1522,21 @@ static int dispatch(const CUtensorMap& map, const DecodeArgs& a, int batch, int 
   return PA_OK;
 }
 
+// Balanced schedule on a pool of 16-token blocks with head dim 64: 32-token
+// tiles of two blocks each (kPagedPairs).
+static int dispatch_pairs(const CUtensorMap& map, const DecodeArgs& a, int batch, int variant, int ctas,
+                          cudaStream_t st) {
+  if (variant == kMma && a.cols > 8) return launch_stream<64, 32, kMma, 0, 2, kPagedPairs>(map, a, batch, ctas, st);
+  if (variant == kMma) return launch_stream<64, 32, kMma, 0, 1, kPagedPairs>(map, a, batch, ctas, st);
+  switch (a.group) {
+    case 1: return launch_stream<64, 32, kCudaCore, 1, 1, kPagedPairs>(map, a, batch, ctas, st);
+    case 2: return launch_stream<64, 32, kCudaCore, 2, 1, kPagedPairs>(map, a, batch, ctas, st);
+    case 4: return launch_stream<64, 32, kCudaCore, 4, 1, kPagedPairs>(map, a, batch, ctas, st);
+    default:
+      return fail(PA_ERR_UNSUPPORTED, "pa_decode: CUDA-core variant has no group size %d", a.group);
+  }
+}
+
 static int decode_impl(pa_bf16* out, const pa_bf16* q, const pa_bf16* kv_pool,
                        const int32_t* block_tables, const int32_t* seq_lens, int batch, int hq,
                        int hkv, int d, int bs, int num_blocks, int max_blocks, int max_seq_len,
@@ -1508,7 +1558,7 @@ static int decode_impl(pa_bf16* out, const pa_bf16* q, const pa_bf16* kv_pool,
   if (!a16(out) || !a16(q) || !a16(kv_pool) || (reinterpret_cast<uintptr_t>(block_tables) & 3u) ||
       (reinterpret_cast<uintptr_t>(seq_lens) & 3u))
     return fail(PA_ERR_INVALID, "pa_decode: misaligned pointer");
-  const bool fused = new_k != nullptr;
+  bool fused = new_k != nullptr;
   if (fused) {
     if (!new_v || !new_slots) return fail(PA_ERR_INVALID, "pa_decode_append: NULL new_v or slot_mapping");
     if (!a16(new_k) || !a16(new_v) || (reinterpret_cast<uintptr_t>(new_slots) & 7u))
@@ -1542,15 +1592,17 @@ static int decode_impl(pa_bf16* out, const pa_bf16* q, const pa_bf16* kv_pool,
   }
   int32_t* err = device_error_word();
   if (err == nullptr) return PA_ERR_CUDA;
+  const bool pairs = plan.stream && stream_tile(d, bs) != bs;
 
   // TMA view of the pool: x = head dim, y = (kv head, row) of one K or V
-  // plane of a block, z = 2*block + (0 keys | 1 values).
+  // plane of a block, z = 2*block + (0 keys | 1 values); a box brings both
+  // planes, or (block pairs) one plane at a time.
   alignas(64) CUtensorMap map;
   const uint64_t dims[3] = {static_cast<uint64_t>(d), static_cast<uint64_t>(hkv) * bs,
                             2ull * static_cast<uint64_t>(num_blocks)};
   const uint64_t strides[2] = {static_cast<uint64_t>(d) * 2,
                                static_cast<uint64_t>(hkv) * bs * d * 2};
-  const uint32_t box[3] = {64u, static_cast<uint32_t>(bs), 2u};
+  const uint32_t box[3] = {64u, static_cast<uint32_t>(bs), pairs ? 1u : 2u};
   rc = encode_tensor_map(&map, 3, const_cast<pa_bf16*>(kv_pool), dims, strides, box, 1);
   if (rc != PA_OK) return rc;
 
@@ -1569,7 +1621,8 @@ static int decode_impl(pa_bf16* out, const pa_bf16* q, const pa_bf16* kv_pool,
   a.group = group;
   a.num_blocks = num_blocks;
   a.max_blocks_per_seq = max_blocks;
-  a.part_blocks = plan.stream ? max_blocks : plan.part_blocks;
+  a.len_cap = pairs ? max_blocks * bs : 0;
+  a.part_blocks = plan.stream ? (pairs ? (max_blocks + 1) / 2 : max_blocks) : plan.part_blocks;
   a.max_parts = plan.max_parts;
   a.scale_log2 = scale * 1.4426950408889634f;
   a.stream_prefix = plan.stream ? reinterpret_cast<int*>(ws + plan.off_prefix) : nullptr;
@@ -1581,7 +1634,7 @@ static int decode_impl(pa_bf16* out, const pa_bf16* q, const pa_bf16* kv_pool,
   a.pool_w = reinterpret_cast<uint4*>(const_cast<pa_bf16*>(kv_pool));
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   if (fused) {
-    if (plan.stream) {  // the decode kernel patches, the merge kernel writes
+    if (plan.stream && !pairs) {  // the decode kernel patches, the merge kernel writes
       a.new_k = reinterpret_cast<const uint4*>(new_k);
       a.new_v = reinterpret_cast<const uint4*>(new_v);
       a.new_slots = new_slots;
@@ -1592,6 +1645,7 @@ static int decode_impl(pa_bf16* out, const pa_bf16* q, const pa_bf16* kv_pool,
     }
   }
 
+  if (pairs) return dispatch_pairs(map, a, batch, variant, plan.ctas, st);
   if (d == 64 && bs == 16) return dispatch<64, 16>(map, a, batch, variant, plan, st);
   if (d == 64 && bs == 32) return dispatch<64, 32>(map, a, batch, variant, plan, st);
   if (d == 128 && bs == 16) return dispatch<128, 16>(map, a, batch, variant, plan, st);

@@ -55,7 +55,7 @@ def test_auto_variant_ragged(d, bs, group):
 @pytest.mark.parametrize("variant,group", [("cuda_core", 1), ("cuda_core", 2), ("cuda_core", 4),
                                            ("mma", 1), ("mma", 2), ("mma", 3), ("mma", 4), ("mma", 5),
                                            ("mma", 8)])
-@pytest.mark.parametrize("d,bs", [(128, 16), (64, 32)])
+@pytest.mark.parametrize("d,bs", [(128, 16), (64, 32), (64, 16)])  # 64/16: two blocks per tile
 @pytest.mark.parametrize("schedule", [pk.PA_SCHEDULE_BALANCED, 0, 64])
 def test_each_variant(variant, group, d, bs, schedule):
     check([5, 31, 33, 200, 480], 2 * group, 2, d, bs, seed=100 + group, variant=variant,

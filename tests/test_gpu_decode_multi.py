@@ -46,7 +46,7 @@ def run_multi(q, pool, tables, lens, scale):
 # the consumer warps pair up, each warp of a pair taking 8 of the columns
 @pytest.mark.parametrize("T,hq,hkv", [(2, 8, 2), (4, 8, 2), (8, 4, 2), (2, 16, 2), (16, 2, 2), (3, 12, 4), (5, 4, 4),
                                       (3, 8, 2), (3, 10, 2)])
-@pytest.mark.parametrize("d,bs", [(128, 16), (64, 32)])
+@pytest.mark.parametrize("d,bs", [(128, 16), (64, 32), (64, 16)])
 def test_multi_matches_oracle(T, hq, hkv, d, bs):
     lens = [T, T + 1, 17, 33, 250, 1000, 2049]
     q, pool, (t_ref, l_ref), (t, l) = make(lens, T, hq, hkv, d, bs, seed=200 + T + hq)
