@@ -319,9 +319,9 @@ def run_gpu(args):
         # allocator work for step i+1 runs while the GPU works on step i
         j = i % INPUT_SETS
         cache.replay_step(j, pending.pop(i))  # upload, decode, output copy: one graph
+        e2e_lens.append(cache.staged("lens", j).numpy().copy())  # bookkeeping while the GPU works
         pending[i + 1] = cache.host_step(ids, (i + 1) % INPUT_SETS)
         stream.synchronize()  # the step's result is on the host
-        e2e_lens.append(cache.staged("lens", j).numpy().copy())
 
     cache.host_step(ids, 0)  # one eager step, then record the graphs on its staged data
     cache.upload(0)
