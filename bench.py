@@ -403,7 +403,7 @@ def run_gpu(args):
                 "d2h_bytes_per_step": int(h_out.nbytes),
                 "ms_per_step": round(e2e_ms / K, 5),
             },
-            "gpu_launches": launches,
+            "gpu_launches": launches * world,  # every rank launches the same kernels
             "clocks": clocks.summary(),
             "device_error_word": dev_err,
         }
