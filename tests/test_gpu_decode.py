@@ -92,6 +92,13 @@ def test_balanced_matches_partition_grid():
     assert (bal.float() - grid.float()).abs().max().item() <= 2 ** -7
 
 
+def test_balanced_schedule_at_its_batch_limit():
+    """4096 requests (the prefix table in shared memory at its largest) on the
+    balanced schedule, short ragged lengths including empty requests."""
+    lens = list(np.random.default_rng(63).integers(0, 40, size=4096))
+    check(lens, 8, 2, 128, 16, seed=63, partition_tokens=pk.PA_SCHEDULE_BALANCED)
+
+
 def test_batch_above_balanced_limit_uses_grid():
     lens = list(np.random.default_rng(62).integers(0, 40, size=4100))
     check(lens, 4, 2, 64, 16, seed=62)
