@@ -147,6 +147,26 @@ def decode_bytes(lens, hq, hkv, d, bs):
     return kv + qo + tables, kv
 
 
+L2_BYTES = 126e6  # B200 L2
+
+
+def l2_note(plan_step, kv_logical, cache):
+    """How the timed steps stand to the L2 (no flush between steps): the K/V
+    a step reads, logically and as distinct physical blocks."""
+    _, _, tables, lens = plan_step
+    nblk = -(-np.asarray(lens, dtype=np.int64) // cache.bs)
+    used = np.unique(np.concatenate([t[:n] for t, n in zip(tables, nblk)]))
+    distinct = len(used) * 2 * cache.hkv * cache.bs * cache.d * 2
+    if distinct > L2_BYTES:
+        return (f"inputs larger than L2, no flush: K/V per step {kv_logical / 1e6:.0f} MB "
+                f"({distinct / 1e6:.0f} MB distinct) > 126 MB")
+    if kv_logical > L2_BYTES:
+        return (f"K/V per step {kv_logical / 1e6:.0f} MB logical but {distinct / 1e6:.0f} MB distinct "
+                f"(shared blocks): blocks read again within a step or the next may come from L2; no flush")
+    return (f"inputs fit in L2 ({kv_logical / 1e6:.1f} MB), no flush: a launch-bound workload, "
+            f"not a bandwidth measurement")
+
+
 def workload_config(name, steps_total, world):
     """The workload fields of the JSON line's ``config``, shared by both arms."""
     p = workloads.plan(name, extra_tokens=steps_total + 1)
@@ -372,7 +392,7 @@ def run_gpu(args):
                 "decode_schedule": (f"balanced persistent: {cache.num_partitions} CTAs"
                                     if cache.schedule == "balanced" else
                                     f"per-partition grid: {cache.num_partitions} partitions"),
-                "l2": f"inputs larger than L2: KV read per step {step_bytes[W][1] / 1e6:.0f} MB > 126 MB",
+                "l2": l2_note(plans[W], step_bytes[W][1], cache),
                 "variant": args.variant,
             },
             "decode_seqs_per_s": round(batch * world * K / (dev_ms * 1e-3), 1),
