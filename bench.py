@@ -578,7 +578,7 @@ def study_memory_waste():
         print(json.dumps(line), flush=True)
 
 
-def study_page_table(iters=30):
+def study_page_table(iters=30, names=("llama8b", "mixed", "long")):
     """pa_decode on the workload's scattered block tables vs on identity
     tables (each request's blocks physically consecutive, same lengths and
     pool format), and vs pa_decode_contiguous on a contiguous reservation per
@@ -591,7 +591,7 @@ def study_page_table(iters=30):
     from paged_kv_cache_354_b200.engine import PagedDecodeCache
 
     dev = torch.device("cuda", torch.cuda.current_device())
-    for name in ("llama8b", "mixed", "long"):
+    for name in names:
         p = workloads.plan(name)
         s = p.shape
         res = {}
@@ -796,6 +796,8 @@ def main():
                     help="decode consumer: auto (tensor cores for GQA groups >= 4), or forced")
     ap.add_argument("--study", choices=["memory-waste", "page-table", "multi-token", "read-bandwidth", "variants"],
                     help="print the study's JSON lines instead of the benchmark line")
+    ap.add_argument("--study-workload", choices=["llama8b", "mixed", "long"], default=None,
+                    help="page-table study: one workload only (default: all three)")
     ap.add_argument("--partition-tokens", type=int, default=0,
                     help="0 = library's choice; -1 = balanced schedule; N > 0 = per-partition grid of "
                          "N-token partitions")
@@ -807,7 +809,7 @@ def main():
     if args.study == "memory-waste":
         study_memory_waste()
     elif args.study == "page-table":
-        study_page_table()
+        study_page_table(names=(args.study_workload,) if args.study_workload else ("llama8b", "mixed", "long"))
     elif args.study == "multi-token":
         study_multi_token()
     elif args.study == "read-bandwidth":
