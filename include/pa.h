@@ -160,7 +160,9 @@ int pa_copy_blocks(pa_bf16* kv_pool, const int32_t* block_pairs, int num_pairs,
  * Other calls use one CTA per (request, KV head, partition of up to 512
  * tokens) and the same kind of merge.
  * Supported: head_dim in {64, 128}; block_size in {16, 32}; num_q_heads a
- * multiple of num_kv_heads with group size 1..8.  Others: PA_ERR_UNSUPPORTED.
+ * multiple of num_kv_heads with group size 1..16 (above 8: the balanced
+ * schedule only -- batch <= 4096, partition_tokens 0 or -1 -- and the
+ * tensor-core variant).  Others: PA_ERR_UNSUPPORTED.
  * Launches: two kernels (decode + merge); the per-partition schedule skips
  * the merge when no request spans two partitions.
  * ------------------------------------------------------------------------ */
@@ -180,7 +182,7 @@ int pa_decode(pa_bf16* out, const pa_bf16* q, const pa_bf16* kv_pool,
 typedef enum pa_decode_variant {
   PA_DECODE_AUTO = 0,      /* tensor cores (mma) for every group: faster at every size measured */
   PA_DECODE_CUDA_CORE = 1, /* fp32 FMA on CUDA cores (group 1, 2 or 4) */
-  PA_DECODE_MMA = 2        /* bf16 mma.sync with fp32 accumulate (group 1..8) */
+  PA_DECODE_MMA = 2        /* bf16 mma.sync with fp32 accumulate (group 1..16) */
 } pa_decode_variant;
 
 /* pa_decode with explicit choices, for measurement and tests.
@@ -303,7 +305,8 @@ int pa_decode_multi(pa_bf16* out, const pa_bf16* q, const pa_bf16* kv_pool,
  * result bit for bit and their timing difference is the cost of paging.
  * max_len must be a positive multiple of 16; seq_lens[b] > max_len is
  * flagged (PA_DEVERR_SEQ_LEN) and clamped.  variant: PA_DECODE_AUTO,
- * PA_DECODE_CUDA_CORE (group 1, 2, 4) or PA_DECODE_MMA.  batch <= 4096.
+ * PA_DECODE_CUDA_CORE (group 1, 2, 4) or PA_DECODE_MMA.  batch <= 4096,
+ * group <= 8.
  * Workspace from pa_decode_contiguous_workspace_size (never 0 bytes).
  * Other arguments as pa_decode.
  * ------------------------------------------------------------------------ */

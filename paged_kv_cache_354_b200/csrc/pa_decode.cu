@@ -1393,7 +1393,11 @@ static int make_plan(int batch, int hq, int hkv, int d, int bs, int max_seq_len,
   const int group = hq / hkv;
   if (qtok > 1 && partition_tokens > 0)
     return fail(PA_ERR_UNSUPPORTED, "multi-token decode runs on the balanced schedule only");
-  if (qtok > 1) partition_tokens = kForceBalanced;
+  // more than 8 (token, head) columns: two MMA tiles on paired warps, which
+  // only the balanced kernel has
+  if (group * qtok > kMaxGroup && partition_tokens > 0)
+    return fail(PA_ERR_UNSUPPORTED, "groups above %d run on the balanced schedule only", kMaxGroup);
+  if (qtok > 1 || group * qtok > kMaxGroup) partition_tokens = kForceBalanced;
   const int sms = sm_count() > 0 ? sm_count() : 148;
   // the balanced schedule pays when there are at least a few tiles per
   // persistent CTA; tiny batches (launch-bound anyway) take the grid
@@ -1450,8 +1454,8 @@ static int check_shape(int batch, int hq, int hkv, int d, int bs, int max_seq_le
                 batch, hq, hkv, max_seq_len);
   if (hq % hkv != 0)
     return fail(PA_ERR_INVALID, "pa_decode: num_q_heads %d not a multiple of num_kv_heads %d", hq, hkv);
-  if (hq / hkv > kMaxGroup)
-    return fail(PA_ERR_UNSUPPORTED, "pa_decode: group size %d above %d", hq / hkv, kMaxGroup);
+  if (hq / hkv > 2 * kMaxGroup)
+    return fail(PA_ERR_UNSUPPORTED, "pa_decode: group size %d above %d", hq / hkv, 2 * kMaxGroup);
   if (d != 64 && d != 128) return fail(PA_ERR_UNSUPPORTED, "pa_decode: head_dim %d not in {64,128}", d);
   if (bs != 16 && bs != 32)
     return fail(PA_ERR_UNSUPPORTED, "pa_decode: block_size %d not in {16,32}", bs);
@@ -1634,7 +1638,9 @@ static int decode_impl(pa_bf16* out, const pa_bf16* q, const pa_bf16* kv_pool,
   a.pool_w = reinterpret_cast<uint4*>(const_cast<pa_bf16*>(kv_pool));
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   if (fused) {
-    if (plan.stream && !pairs) {  // the decode kernel patches, the merge kernel writes
+    // the decode kernel patches the staged tile, the merge kernel stores the
+    // row; with block pairs or paired warps the cache write runs first
+    if (plan.stream && !pairs && a.cols <= kMaxGroup) {
       a.new_k = reinterpret_cast<const uint4*>(new_k);
       a.new_v = reinterpret_cast<const uint4*>(new_v);
       a.new_slots = new_slots;
@@ -1677,6 +1683,8 @@ static int contiguous_plan(int batch, int hq, int hkv, int d, int max_len, Plan*
   if (max_len <= 0 || max_len % kContiguousTile != 0)
     return fail(PA_ERR_INVALID, "pa_decode_contiguous: max_len %d not a positive multiple of %d", max_len,
                 kContiguousTile);
+  if (hq / hkv > kMaxGroup)
+    return fail(PA_ERR_UNSUPPORTED, "pa_decode_contiguous: group size %d above %d", hq / hkv, kMaxGroup);
   return make_plan(batch, hq, hkv, d, kContiguousTile, max_len, kForceBalanced, plan);
 }
 

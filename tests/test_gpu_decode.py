@@ -92,6 +92,14 @@ def test_balanced_matches_partition_grid():
     assert (bal.float() - grid.float()).abs().max().item() <= 2 ** -7
 
 
+@pytest.mark.parametrize("d,bs", [(128, 16), (64, 32), (64, 16)])
+@pytest.mark.parametrize("schedule", [0, pk.PA_SCHEDULE_BALANCED])
+def test_group_16(d, bs, schedule):
+    """16 query heads per KV head: two 8-wide MMA tiles on paired warps
+    (balanced schedule only)."""
+    check(RAGGED, 32, 2, d, bs, seed=70 + d + bs, partition_tokens=schedule)
+
+
 def test_balanced_schedule_at_its_batch_limit():
     """4096 requests (the prefix table in shared memory at its largest) on the
     balanced schedule, short ragged lengths including empty requests."""

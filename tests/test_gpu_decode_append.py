@@ -27,6 +27,7 @@ def bits(t):
     ([900, 33, 5, 2047, 400], 16, 4, 64, 32),                      # balanced, other shape
     ([3, 20, 1], 4, 4, 64, 16),                                    # little work: per-partition grid
     ([900, 33, 5, 2047, 400, 1600, 2500, 3000], 16, 4, 64, 16),   # balanced on block pairs: write, then decode
+    ([700, 1, 2049, 64, 300, 1500, 17, 1024], 32, 2, 128, 16),    # group 16 (paired warps): write, then decode
 ])
 def test_append_equals_separate_calls(lens, hq, hkv, d, bs):
     dev = torch.device("cuda", torch.cuda.current_device())
