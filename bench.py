@@ -714,7 +714,8 @@ def study_multi_token(iters=30):
 def study_variants(iters=20):
     """Tensor-core vs CUDA-core consumer across GQA group sizes: pa_decode on
     the llama8b lengths and shuffled pool, Hkv in {8, 32}, head dim 128 and
-    (Hkv 8) 64, groups 1, 2, 4, 8; CUDA events over back-to-back launches."""
+    (Hkv 8) 64, groups 1, 2, 4, 8, 16, 32 (CUDA cores: 1, 2, 4); CUDA events
+    over back-to-back launches."""
     import torch
 
     import paged_kv_cache_354_b200 as pk
@@ -731,7 +732,7 @@ def study_variants(iters=20):
         ids = workloads.populate(alloc, p)
         tables, lens = alloc.block_tables(ids, -(-int(max(p.seq_lens)) // bs))
         d_t, d_l = torch.as_tensor(tables, device=dev), torch.as_tensor(lens, device=dev)
-        for g in (1, 2, 4, 8):
+        for g in (1, 2, 4, 8, 16, 32):
             q = torch.randn((len(ids), hkv * g, d), generator=gen, device=dev).bfloat16()
             out = torch.empty_like(q)
             nbytes = decode_bytes(lens, hkv * g, hkv, d, bs)[0]

@@ -160,7 +160,7 @@ int pa_copy_blocks(pa_bf16* kv_pool, const int32_t* block_pairs, int num_pairs,
  * Other calls use one CTA per (request, KV head, partition of up to 512
  * tokens) and the same kind of merge.
  * Supported: head_dim in {64, 128}; block_size in {16, 32}; num_q_heads a
- * multiple of num_kv_heads with group size 1..16 (above 8: the balanced
+ * multiple of num_kv_heads with group size 1..32 (above 8: the balanced
  * schedule only -- batch <= 4096, partition_tokens 0 or -1 -- and the
  * tensor-core variant).  Others: PA_ERR_UNSUPPORTED.
  * Launches: two kernels (decode + merge); the per-partition schedule skips
@@ -182,7 +182,7 @@ int pa_decode(pa_bf16* out, const pa_bf16* q, const pa_bf16* kv_pool,
 typedef enum pa_decode_variant {
   PA_DECODE_AUTO = 0,      /* tensor cores (mma) for every group: faster at every size measured */
   PA_DECODE_CUDA_CORE = 1, /* fp32 FMA on CUDA cores (group 1, 2 or 4) */
-  PA_DECODE_MMA = 2        /* bf16 mma.sync with fp32 accumulate (group 1..16) */
+  PA_DECODE_MMA = 2        /* bf16 mma.sync with fp32 accumulate (group 1..32) */
 } pa_decode_variant;
 
 /* pa_decode with explicit choices, for measurement and tests.
@@ -273,7 +273,7 @@ int pa_decode_append(pa_bf16* out, const pa_bf16* q, pa_bf16* kv_pool, const pa_
  * out = 0.
  *
  * q, out       : device bf16 [batch][T][num_q_heads][head_dim]
- * Other arguments as pa_decode.  (num_q_heads / num_kv_heads) * T <= 16.
+ * Other arguments as pa_decode.  (num_q_heads / num_kv_heads) * T <= 32.
  * Always the balanced schedule (batch <= 4096) and the tensor-core
  * consumer; workspace from pa_decode_multi_workspace_size.
  * ------------------------------------------------------------------------ */

@@ -752,13 +752,15 @@ constexpr int kStreamCtasPerSm = PA_STREAM_CTAS_PER_SM;
 constexpr int kStreamMaxBatch = 4096;  // the prefix table lives in shared memory
 
 // Consumer groups of the balanced kernel: with up to 8 (token, head) columns
-// each consumer warp takes every fourth block alone; with 16 (two 8-wide MMA
-// tiles) the warps pair up, both warps of a pair take every other block and
-// each computes 8 of the columns, so no warp carries the 16-column tile's
-// registers and every pair keeps twice as many stages in flight.
+// each consumer warp takes every fourth block alone; with up to 16 (two
+// 8-wide MMA tiles) the warps pair up, both warps of a pair take every other
+// block and each computes 8 of the columns; with up to 32 all four warps take
+// every block, 8 columns each.  No warp carries more than one tile's
+// registers, and a group keeps kStages / kGroups stages in flight.
 template <int NT>
 struct StreamGroups {
-  static constexpr int kPerGroup = NT == 2 ? 2 : 1;          // warps sharing a block
+  static_assert(NT == 1 || NT == 2 || NT == 4, "1, 2 or 4 tiles of 8 columns");
+  static constexpr int kPerGroup = NT;                         // warps sharing a block
   static constexpr int kGroups = kConsumerWarps / kPerGroup;  // block streams per CTA
 };
 
@@ -1039,7 +1041,7 @@ __global__ void __launch_bounds__(kThreads, kStreamCtasPerSm)
     const int cols = a.cols;
     const size_t q_tok_stride = static_cast<size_t>(a.num_q_heads) * D;
     const int grp_id = warp / grp::kPerGroup;  // block stream of this warp
-    const int sub = warp % grp::kPerGroup;     // its 8 columns within the group's 16
+    const int sub = warp % grp::kPerGroup;     // its 8 columns within the group's
     int b, h, k;
     stream_locate(prefix, batch, hkv, u_begin, b, h, k);
     long long u = u_begin;
@@ -1118,7 +1120,7 @@ __global__ void __launch_bounds__(kThreads, kStreamCtasPerSm)
         for (int idx = threadIdx.x; idx < cols * D / 2; idx += kConsumerWarps * 32) {
           const int c = (2 * idx) / D;  // column: token c / g, head c % g
           const int d = (2 * idx) % D;
-          const int csub = grp::kPerGroup == 2 ? (c >> 3) : 0;  // which member of a group
+          const int csub = grp::kPerGroup > 1 ? (c >> 3) : 0;  // which member of a group
           const int cr = c - 8 * csub;                           // row in that member's scratch
           float mm = -INFINITY;
 #pragma unroll
@@ -1393,8 +1395,8 @@ static int make_plan(int batch, int hq, int hkv, int d, int bs, int max_seq_len,
   const int group = hq / hkv;
   if (qtok > 1 && partition_tokens > 0)
     return fail(PA_ERR_UNSUPPORTED, "multi-token decode runs on the balanced schedule only");
-  // more than 8 (token, head) columns: two MMA tiles on paired warps, which
-  // only the balanced kernel has
+  // more than 8 (token, head) columns: two or four MMA tiles on grouped
+  // warps, which only the balanced kernel has
   if (group * qtok > kMaxGroup && partition_tokens > 0)
     return fail(PA_ERR_UNSUPPORTED, "groups above %d run on the balanced schedule only", kMaxGroup);
   if (qtok > 1 || group * qtok > kMaxGroup) partition_tokens = kForceBalanced;
@@ -1454,8 +1456,8 @@ static int check_shape(int batch, int hq, int hkv, int d, int bs, int max_seq_le
                 batch, hq, hkv, max_seq_len);
   if (hq % hkv != 0)
     return fail(PA_ERR_INVALID, "pa_decode: num_q_heads %d not a multiple of num_kv_heads %d", hq, hkv);
-  if (hq / hkv > 2 * kMaxGroup)
-    return fail(PA_ERR_UNSUPPORTED, "pa_decode: group size %d above %d", hq / hkv, 2 * kMaxGroup);
+  if (hq / hkv > 4 * kMaxGroup)
+    return fail(PA_ERR_UNSUPPORTED, "pa_decode: group size %d above %d", hq / hkv, 4 * kMaxGroup);
   if (d != 64 && d != 128) return fail(PA_ERR_UNSUPPORTED, "pa_decode: head_dim %d not in {64,128}", d);
   if (bs != 16 && bs != 32)
     return fail(PA_ERR_UNSUPPORTED, "pa_decode: block_size %d not in {16,32}", bs);
@@ -1495,6 +1497,7 @@ template <int D, int BS>
 static int dispatch(const CUtensorMap& map, const DecodeArgs& a, int batch, int variant,
                     const Plan& plan, cudaStream_t st) {
   if (plan.stream) {
+    if (variant == kMma && a.cols > 16) return launch_stream<D, BS, kMma, 0, 4>(map, a, batch, plan.ctas, st);
     if (variant == kMma && a.cols > 8) return launch_stream<D, BS, kMma, 0, 2>(map, a, batch, plan.ctas, st);
     if (variant == kMma) return launch_stream<D, BS, kMma, 0, 1>(map, a, batch, plan.ctas, st);
     switch (a.group) {
@@ -1530,6 +1533,7 @@ static int dispatch(const CUtensorMap& map, const DecodeArgs& a, int batch, int 
 // tiles of two blocks each (kPagedPairs).
 static int dispatch_pairs(const CUtensorMap& map, const DecodeArgs& a, int batch, int variant, int ctas,
                           cudaStream_t st) {
+  if (variant == kMma && a.cols > 16) return launch_stream<64, 32, kMma, 0, 4, kPagedPairs>(map, a, batch, ctas, st);
   if (variant == kMma && a.cols > 8) return launch_stream<64, 32, kMma, 0, 2, kPagedPairs>(map, a, batch, ctas, st);
   if (variant == kMma) return launch_stream<64, 32, kMma, 0, 1, kPagedPairs>(map, a, batch, ctas, st);
   switch (a.group) {
@@ -1571,9 +1575,9 @@ static int decode_impl(pa_bf16* out, const pa_bf16* q, const pa_bf16* kv_pool,
   }
   const int group = hq / hkv;
   if (qtok < 1) return fail(PA_ERR_INVALID, "num_query_tokens %d below 1", qtok);
-  if (group * qtok > 2 * kMaxGroup)
+  if (group * qtok > 4 * kMaxGroup)
     return fail(PA_ERR_UNSUPPORTED, "group %d x query tokens %d above %d columns", group, qtok,
-                2 * kMaxGroup);
+                4 * kMaxGroup);
   if (qtok > 1 && variant == kCudaCore)
     return fail(PA_ERR_UNSUPPORTED, "multi-token decode has the tensor-core variant only");
   // tensor cores for every group: at scale they beat the CUDA-core consumer
@@ -1787,8 +1791,8 @@ int pa_decode_multi_workspace_size(int batch, int num_query_tokens, int num_q_he
   int rc = check_shape(batch, num_q_heads, num_kv_heads, head_dim, block_size, max_seq_len);
   if (rc != PA_OK) return rc;
   if (num_query_tokens < 1) return fail(PA_ERR_INVALID, "num_query_tokens %d below 1", num_query_tokens);
-  if (num_q_heads / num_kv_heads * num_query_tokens > 2 * kMaxGroup)
-    return fail(PA_ERR_UNSUPPORTED, "group x query tokens above %d columns", 2 * kMaxGroup);
+  if (num_q_heads / num_kv_heads * num_query_tokens > 4 * kMaxGroup)
+    return fail(PA_ERR_UNSUPPORTED, "group x query tokens above %d columns", 4 * kMaxGroup);
   Plan plan;
   rc = make_plan(batch, num_q_heads, num_kv_heads, head_dim, block_size, max_seq_len, kForceBalanced,
                  &plan, num_query_tokens);

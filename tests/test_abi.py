@@ -61,8 +61,8 @@ def test_invalid_arguments_fail_before_launch():
         pk.PA_ERR_UNSUPPORTED
     assert lib.pa_decode_workspace_size(4, 8, 2, 128, 8, 100, ctypes.byref(nb), ctypes.byref(parts)) == \
         pk.PA_ERR_UNSUPPORTED
-    assert lib.pa_decode_workspace_size(4, 34, 2, 128, 16, 100, ctypes.byref(nb), ctypes.byref(parts)) == \
-        pk.PA_ERR_UNSUPPORTED  # group 17
+    assert lib.pa_decode_workspace_size(4, 66, 2, 128, 16, 100, ctypes.byref(nb), ctypes.byref(parts)) == \
+        pk.PA_ERR_UNSUPPORTED  # group 33
     # groups above 8 run on the balanced schedule only
     assert lib.pa_decode_workspace_size_ex(4, 32, 2, 128, 16, 1000, 256, ctypes.byref(nb),
                                            ctypes.byref(parts), None) == pk.PA_ERR_UNSUPPORTED

@@ -94,10 +94,11 @@ def test_balanced_matches_partition_grid():
 
 @pytest.mark.parametrize("d,bs", [(128, 16), (64, 32), (64, 16)])
 @pytest.mark.parametrize("schedule", [0, pk.PA_SCHEDULE_BALANCED])
-def test_group_16(d, bs, schedule):
-    """16 query heads per KV head: two 8-wide MMA tiles on paired warps
-    (balanced schedule only)."""
-    check(RAGGED, 32, 2, d, bs, seed=70 + d + bs, partition_tokens=schedule)
+@pytest.mark.parametrize("hq,hkv", [(32, 2), (24, 2), (64, 2), (32, 1)])
+def test_wide_groups(d, bs, schedule, hq, hkv):
+    """Groups of 12, 16 and 32 query heads per KV head (32/1: multi-query):
+    two or four 8-wide MMA tiles on grouped warps (balanced schedule only)."""
+    check(RAGGED, hq, hkv, d, bs, seed=70 + d + bs + hq, partition_tokens=schedule)
 
 
 def test_balanced_schedule_at_its_batch_limit():
