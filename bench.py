@@ -256,87 +256,125 @@ def combine_ranks(times_ms, totals, device, world):
     return tuple(t.tolist()) + tuple(w.tolist())
 
 
-def run_gpu(args):
+MIN_TIMED_S = 0.5  # device time each timed loop reaches (the clock record needs it)
+OTHER_WORKLOADS = ("long", "beam", "mixed", "tiny")
+
+
+def repeats_for(est_ms, units, min_s):
+    """Repetitions of a loop of ``units`` items of ``est_ms`` each that reach
+    ``min_s`` of device time."""
+    if est_ms <= 0:
+        return 1
+    return max(1, int(math.ceil(min_s * 1e3 / (est_ms * units))))
+
+
+def timed_ms(stream, fn):
+    """Device time of ``fn``'s launches: CUDA events on the launching stream,
+    synchronised on both sides."""
+    import torch
+
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    fn()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    return e0.elapsed_time(e1)
+
+
+def agree_max(x, device, world):
+    """The largest of every rank's x (so all ranks repeat a loop equally often)."""
     import torch
     import torch.distributed as dist
 
-    world = int(os.environ.get("WORLD_SIZE", "1"))
-    rank = int(os.environ.get("RANK", "0"))
-    local = int(os.environ.get("LOCAL_RANK", "0"))
-    if world > 1:
-        torch.cuda.set_device(local)
-        dist.init_process_group("nccl", timeout=__import__("datetime").timedelta(seconds=120))
-    device = torch.device("cuda", local if world > 1 else torch.cuda.current_device())
-    torch.cuda.set_device(device)
-    from paged_kv_cache_354_b200 import pa_device_error
+    if world == 1:
+        return x
+    t = torch.tensor([float(x)], device=device, dtype=torch.float64)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return int(t.item())
 
-    K, W = args.steps, args.warmup
-    variant = {"auto": 0, "cuda_core": 1, "mma": 2}[args.variant]
-    p, cache, ids, gen = build_cache(args.workload, 2 * (W + K) + 4, rank, device, variant=variant,
-                                     partition_tokens=args.partition_tokens)
+
+def device_arm(name, K, W, rank, device, world, variant=0, partition_tokens=0, min_s=MIN_TIMED_S):
+    """Device-timed figures of one workload, every input resident in HBM.
+
+    Steps: W warm-up steps, then the same K steps (copy-on-write copies, the
+    fused cache write + decode + merge of one new token per request) repeated
+    R times so the timed region holds at least ``min_s`` of device time.
+    Decode alone: back-to-back pa_decode launches (main kernel + merge) on
+    the last step's inputs, repeated likewise.  Clocks are sampled over both
+    timed loops."""
+    import torch
+    import torch.distributed as dist
+
+    p, cache, ids, gen = build_cache(name, 2 * (W + K) + 4, rank, device, variant=variant,
+                                     partition_tokens=partition_tokens)
     batch = len(ids)
     qs, ks, vs = make_inputs(cache, batch, gen, device)
     out = torch.empty_like(qs[0])
     stream = torch.cuda.current_stream()
-
-    # ---- device-timed arm: all step metadata precomputed and resident
     plans = [cache.plan_append(ids) for _ in range(W + K)]
     d_slots = [torch.as_tensor(pl[0], device=device) for pl in plans]
     d_pairs = [torch.as_tensor(pl[1].reshape(-1, 2), device=device) for pl in plans]
     d_tables = [torch.as_tensor(pl[2], device=device) for pl in plans]
     d_lens = [torch.as_tensor(pl[3], device=device) for pl in plans]
     step_bytes = [decode_bytes(pl[3], cache.hq, cache.hkv, cache.d, cache.bs) for pl in plans]
-    launches = sum(cache.launches_per_step(len(pl[1])) for pl in plans[W:])
 
     def dev_step(i):
         j = i % INPUT_SETS
         cache.run(qs[j], ks[j], vs[j], out, d_slots[i], d_tables[i], d_lens[i], d_pairs[i])
 
-    for i in range(W):
-        dev_step(i)
-    torch.cuda.synchronize()
-    if world > 1:
-        dist.barrier()
-    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    with ClockSampler(device.index) as clocks:
-        start.record(stream)
-        for i in range(W, W + K):
-            j = i % INPUT_SETS
-            cache.run(qs[j], ks[j], vs[j], out, d_slots[i], d_tables[i], d_lens[i], d_pairs[i])
-        end.record(stream)
-        torch.cuda.synchronize()
-        # the dominant kernel alone: K back-to-back decode launches (main + merge)
-        # on the last step's inputs, bracketed by events on the launching stream
-        k0, k1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        last = W + K - 1
-        k0.record(stream)
-        for i in range(K):
-            cache.decode(qs[i % INPUT_SETS], out, d_tables[last], d_lens[last])
-        k1.record(stream)
-        torch.cuda.synchronize()
-    if world > 1:
-        dist.barrier()
-    dev_ms = start.elapsed_time(end)
-    decode_ms = [k0.elapsed_time(k1) / K]
-    decode_bytes_last = step_bytes[last][0]
-    bytes_timed = sum(b for b, _ in step_bytes[W:])
-    kv_timed = sum(kv for _, kv in step_bytes[W:])
+    last = W + K - 1
 
-    # ---- end-to-end arm: per step the host allocator writes the step's
-    # metadata into a pinned staging buffer that already holds the step's
-    # q/k/v; one CUDA graph then copies it to the device, runs the fused
-    # cache write + decode + merge and copies the output back
+    def decode_once(i):
+        cache.decode(qs[i % INPUT_SETS], out, d_tables[last], d_lens[last])
+
+    est_step = timed_ms(stream, lambda: [dev_step(i) for i in range(W)]) / W
+    est_dec = timed_ms(stream, lambda: [decode_once(i) for i in range(3)]) / 3
+    R = agree_max(repeats_for(est_step, K, min_s), device, world)
+    Rd = agree_max(repeats_for(est_dec, K, min_s), device, world)
+    if world > 1:
+        dist.barrier()
+    with ClockSampler(device.index) as clocks:
+        step_ms = timed_ms(stream, lambda: [dev_step(i) for _ in range(R) for i in range(W, W + K)])
+        dec_ms = timed_ms(stream, lambda: [decode_once(i) for i in range(Rd * K)])
+    if world > 1:
+        dist.barrier()
+    merge = 1 if (cache.schedule == "balanced" or cache.num_partitions > 1) else 0
+    return {
+        "p": p, "cache": cache, "ids": ids, "gen": gen, "qs": qs, "ks": ks, "vs": vs, "out": out,
+        "plans": plans, "step_bytes": step_bytes, "R": R, "Rd": Rd,
+        "step_ms": step_ms, "steps_timed": R * K,
+        "bytes_timed": R * sum(b for b, _ in step_bytes[W:]),
+        "kv_timed": R * sum(kv for _, kv in step_bytes[W:]),
+        "decode_ms": dec_ms / (Rd * K), "decode_bytes": step_bytes[last][0],
+        "launches": R * sum(cache.launches_per_step(len(pl[1])) for pl in plans[W:]),
+        "decode_launches": Rd * K * (1 + merge),
+        "clocks": clocks.summary(),
+    }
+
+
+def e2e_arm(arm, K, W, device, world):
+    """End to end through the engine, K steps: per step the host allocator
+    writes the step's metadata into a pinned staging buffer that already
+    holds the step's q/k/v; one CUDA graph copies it to the device, runs the
+    fused cache write + decode + merge and copies the output back; the
+    allocator work for step i+1 runs on the host while the GPU works on
+    step i; the host waits for step i's output before going on."""
+    import torch
+    import torch.distributed as dist
+
+    cache, ids, out = arm["cache"], arm["ids"], arm["out"]
+    stream = torch.cuda.current_stream()
     for j in range(INPUT_SETS):
-        cache.staged("q", j).copy_(qs[j].cpu())
-        cache.staged("k", j).copy_(ks[j].cpu())
-        cache.staged("v", j).copy_(vs[j].cpu())
+        cache.staged("q", j).copy_(arm["qs"][j].cpu())
+        cache.staged("k", j).copy_(arm["ks"][j].cpu())
+        cache.staged("v", j).copy_(arm["vs"][j].cpu())
     h_out = torch.empty(out.shape, dtype=out.dtype).pin_memory()
     e2e_lens = []
     pending = {}
 
     def e2e_step(i):
-        # step i's metadata was staged in buffer j during step i-1; the
-        # allocator work for step i+1 runs while the GPU works on step i
+        # step i's metadata was staged in buffer j during step i-1
         j = i % INPUT_SETS
         cache.replay_step(j, pending.pop(i))  # upload, decode, output copy: one graph
         e2e_lens.append(cache.staged("lens", j).numpy().copy())  # bookkeeping while the GPU works
@@ -354,25 +392,89 @@ def run_gpu(args):
     if world > 1:
         dist.barrier()
     e2e_lens.clear()
-    e_start, e_end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    e_start.record(stream)
-    for i in range(K):
-        e2e_step(W + i)
-    e_end.record(stream)
-    torch.cuda.synchronize()
-    e2e_ms = e_start.elapsed_time(e_end)
-    e2e_bytes = sum(decode_bytes(ln, cache.hq, cache.hkv, cache.d, cache.bs)[0] for ln in e2e_lens)
-    e2e_h2d = K * cache.stage_bytes
+    ms = timed_ms(stream, lambda: [e2e_step(W + i) for i in range(K)])
+    nbytes = sum(decode_bytes(ln, cache.hq, cache.hkv, cache.d, cache.bs)[0] for ln in e2e_lens)
+    return ms, nbytes, cache.stage_bytes, int(h_out.nbytes)
+
+
+def workload_entry(name, arm, peaks, world):
+    """One workload's device-timed figures for the JSON line."""
+    step_gbs = arm["bytes_timed"] / (arm["step_ms"] * 1e-3) / 1e9
+    dec_gbs = arm["decode_bytes"] / (arm["decode_ms"] * 1e-3) / 1e9
+    cache = arm["cache"]
+    return {
+        "workload": workload_config(name, 0, world)["workload"],
+        "step_gbs": round(step_gbs, 2),
+        "step_ms": round(arm["step_ms"] / arm["steps_timed"], 5),
+        "step_frac_of_hbm_peak": round(step_gbs / peaks["hbm_gbs"], 4),
+        "decode_gbs": round(dec_gbs, 2),
+        "decode_ms": round(arm["decode_ms"], 5),
+        "decode_frac_of_hbm_peak": round(dec_gbs / peaks["hbm_gbs"], 4),
+        "decode_seqs_per_s": round(len(arm["ids"]) / (arm["step_ms"] / arm["steps_timed"] * 1e-3), 1),
+        "steps_timed": arm["steps_timed"],
+        "decode_launches_timed": arm["Rd"],
+        "decode_schedule": (f"balanced persistent: {cache.num_partitions} CTAs"
+                            if cache.schedule == "balanced" else
+                            f"per-partition grid: {cache.num_partitions} partitions"),
+        "l2": l2_note(arm["plans"][-1], arm["step_bytes"][-1][1], cache),
+        "clocks": arm["clocks"],
+    }
+
+
+def run_gpu(args):
+    import torch
+    import torch.distributed as dist
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=__import__("datetime").timedelta(seconds=120))
+    device = torch.device("cuda", local if world > 1 else torch.cuda.current_device())
+    torch.cuda.set_device(device)
+    from paged_kv_cache_354_b200 import pa_device_error
+
+    K, W = args.steps, args.warmup
+    variant = {"auto": 0, "cuda_core": 1, "mma": 2}[args.variant]
+    arm = device_arm(args.workload, K, W, rank, device, world, variant, args.partition_tokens, args.min_seconds)
+    e2e_ms, e2e_bytes, stage_bytes, d2h_bytes = e2e_arm(arm, K, W, device, world)
     dev_err = pa_device_error()
 
     # ---- max over ranks (times), sum over ranks (work)
-    dev_ms, e2e_ms, decode_avg_ms, bytes_all, e2e_bytes_all, kv_all = combine_ranks(
-        [dev_ms, e2e_ms, float(np.mean(decode_ms))], [bytes_timed, e2e_bytes, kv_timed], device, world)
+    step_ms, e2e_ms, decode_ms, bytes_all, e2e_bytes_all, kv_all = combine_ranks(
+        [arm["step_ms"], e2e_ms, arm["decode_ms"]], [arm["bytes_timed"], e2e_bytes, arm["kv_timed"]], device,
+        world)
+    cache, steps_timed = arm["cache"], arm["steps_timed"]
+    batch = len(arm["ids"])
+    summary = {
+        "mean_seq_len": round(float(np.mean(arm["plans"][W][3])), 1),
+        "decode_schedule": (f"balanced persistent: {cache.num_partitions} CTAs"
+                            if cache.schedule == "balanced" else
+                            f"per-partition grid: {cache.num_partitions} partitions"),
+        "l2": l2_note(arm["plans"][W], arm["step_bytes"][W][1], cache),
+        "variant": args.variant,
+    }
+    launches, dec_launches, decode_bytes_last = arm["launches"], arm["decode_launches"], arm["decode_bytes"]
+    clocks = arm["clocks"]
+    del arm, cache
+    torch.cuda.empty_cache()
+
+    # ---- the other workloads, device-timed (one GPU, default workload only)
+    others = {}
+    if world == 1 and args.workload == "llama8b" and not args.no_workloads:
+        peaks = load_peaks()
+        for name in OTHER_WORKLOADS:
+            o = device_arm(name, K, W, rank, device, world, min_s=args.min_seconds / 2)
+            others[name] = workload_entry(name, o, peaks, world)
+            del o
+            torch.cuda.empty_cache()
+        dev_err |= pa_device_error()
 
     if rank == 0:
         peaks = load_peaks()
-        gbs = bytes_all / (dev_ms * 1e-3) / 1e9
-        achieved = decode_bytes_last / (decode_avg_ms * 1e-3) / 1e9
+        gbs = bytes_all / (step_ms * 1e-3) / 1e9
+        achieved = decode_bytes_last / (decode_ms * 1e-3) / 1e9
         line = {
             "metric": METRIC,
             "value": round(gbs, 2),
@@ -380,29 +482,25 @@ def run_gpu(args):
             "n_gpus": world,
             "steps": K,
             "warmup": W,
-            "ms_per_step": round(dev_ms / K, 5),
+            "ms_per_step": round(step_ms / steps_timed, 5),
             "higher_is_better": True,
             "scaling": "weak",
             "vs_baseline": None,
             "dtype": "bf16",
             "data": "synthetic (seeded bf16 N(0,1) q/K/V; seeded lengths and shuffled block pool)",
-            "config": {
-                **workload_config(args.workload, 2 * (W + K) + 4, world),
-                "mean_seq_len": round(float(np.mean(plans[W][3])), 1),
-                "decode_schedule": (f"balanced persistent: {cache.num_partitions} CTAs"
-                                    if cache.schedule == "balanced" else
-                                    f"per-partition grid: {cache.num_partitions} partitions"),
-                "l2": l2_note(plans[W], step_bytes[W][1], cache),
-                "variant": args.variant,
-            },
-            "decode_seqs_per_s": round(batch * world * K / (dev_ms * 1e-3), 1),
+            "config": workload_config(args.workload, 2 * (W + K) + 4, world),
+            "run": {**summary, "timed_repeats": steps_timed // K, "steps_timed": steps_timed,
+                    "timing": "the K steps repeated timed_repeats times back to back (each repetition the same "
+                              "K steps: copy-on-write copies, fused cache write + decode + merge); one pair of "
+                              "CUDA events around all of them; ms_per_step = their device time / steps_timed"},
+            "decode_seqs_per_s": round(batch * world * steps_timed / (step_ms * 1e-3), 1),
             "frac_of_hbm_peak": round(gbs / world / peaks["hbm_gbs"], 4),
             # against the B200 data-sheet bandwidth (8 TB/s) rather than the measured copy
             "frac_of_spec_hbm": round(gbs / world / SPEC_HBM_GBS, 4),
             "spec_hbm_gbs": SPEC_HBM_GBS,
             "roofline": {
                 "bound": "hbm",
-                "kernel": "pa_decode (main + split-K merge), K back-to-back launches",
+                "kernel": "pa_decode (main + split-K merge), back-to-back launches",
                 "achieved": round(achieved, 2),
                 "peak": peaks["hbm_gbs"],
                 "unit": "GB/s",
@@ -410,23 +508,27 @@ def run_gpu(args):
                 "peak_source": peaks["source"],
                 "traffic": captured_traffic(args.workload, args.variant, args.partition_tokens),
                 "traffic_note": "dram read+write per launch of the main decode kernel from the committed "
-                                "ncu capture; null when none matches the current source",
+                                "ncu capture; null unless that capture was taken on the current decode sources",
+                "launches_timed": dec_launches,
             },
             "e2e": {
                 "value": round(e2e_bytes_all / (e2e_ms * 1e-3) / 1e9, 2),
                 "unit": "GB/s",
-                "h2d_bytes_per_step": int(e2e_h2d / K),
+                "h2d_bytes_per_step": int(stage_bytes),
+                "d2h_bytes_per_step": int(d2h_bytes),
+                "ms_per_step": round(e2e_ms / K, 5),
+                "steps_timed": K,
                 "path": "per step: one CUDA graph holding the H2D copy of a pinned staging buffer "
                         "(metadata from the C++ allocator + the step's q/k/v), the fused cache write + "
                         "decode + merge and the D2H copy of the output; then a sync; the allocator work "
                         "for the next step runs on the host while the GPU works",
-                "d2h_bytes_per_step": int(h_out.nbytes),
-                "ms_per_step": round(e2e_ms / K, 5),
             },
-            "gpu_launches": launches * world,  # every rank launches the same kernels
-            "clocks": clocks.summary(),
+            "gpu_launches": launches * world,  # the step loop (value's timed region), every rank
+            "clocks": clocks,
             "device_error_word": dev_err,
         }
+        if others:
+            line["workloads"] = others
         if world == 1 and not args.no_cpu_baseline:
             line["cpu_baseline"] = cpu_baseline(args.workload, args.cpu_seconds)
         print(json.dumps(line), flush=True)
@@ -527,9 +629,9 @@ def run_reference(args):
         "vs_baseline": None,
         "dtype": "f64",
         "data": "synthetic (seeded bf16 N(0,1) K/V and q, upcast to f64)",
-        "config": {**workload_config(args.workload, 2 * (args.warmup + args.steps) + 4,
-                                     int(os.environ.get("WORLD_SIZE", "1"))),
-                   "note": "each step decodes at least one whole request of the workload on the host"},
+        "config": workload_config(args.workload, 2 * (args.warmup + args.steps) + 4,
+                                  int(os.environ.get("WORLD_SIZE", "1"))),
+        "run": {"note": "each step decodes at least one whole request of the workload on the host"},
         "cpu_baseline": {"value": round(value, 4), "unit": "GB/s", "cores": 1, "kind": "oracle",
                          "sample": runner.describe(n)},
         "e2e": {"value": round(value, 4), "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
@@ -803,6 +905,10 @@ def main():
                     help="0 = library's choice; -1 = balanced schedule; N > 0 = per-partition grid of "
                          "N-token partitions")
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
+    ap.add_argument("--min-seconds", type=float, default=MIN_TIMED_S,
+                    help="device time each timed loop reaches (the K steps are repeated until it does)")
+    ap.add_argument("--no-workloads", action="store_true",
+                    help="skip the device-timed figures of the other workloads")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     args = ap.parse_args()
     if args.warmup < 3:

@@ -142,7 +142,8 @@ int pa_copy_blocks(pa_bf16* kv_pool, const int32_t* block_pairs, int num_pairs,
  *                length inside its last block may hold anything (even NaN).
  * block_tables : device int32 [batch][max_blocks_per_seq]; only the first
  *                ceil(seq_len/block_size) entries of a row are read.  An
- *                entry outside [0, num_blocks) reads zeros and flags
+ *                entry outside [0, num_blocks) reads as a block of zeros
+ *                (its positions take part with logit 0) and flags
  *                PA_DEVERR_BLOCK_ID.
  * seq_lens     : device int32 [batch]; 0 <= seq_len <= max_seq_len.  A value
  *                beyond max_blocks_per_seq*block_size is clamped and flags

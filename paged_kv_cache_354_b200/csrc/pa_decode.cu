@@ -604,7 +604,7 @@ __global__ void __launch_bounds__(kThreads, (VAR == kMma || G <= 2) ? 3 : 2)
         phys = __ldg(trow + base + lane);
         if (static_cast<unsigned>(phys) >= static_cast<unsigned>(a.num_blocks)) {
           flag_error(a.err, PA_DEVERR_BLOCK_ID);
-          phys = 0;  // read a valid block instead; the result is flagged as wrong
+          phys = a.num_blocks;  // past the tensor map: TMA fills the tile with zeros
         }
       }
       const int cnt = min(32, n - base);
@@ -975,7 +975,7 @@ __global__ void __launch_bounds__(kThreads, kStreamCtasPerSm)
             phys = __ldg(trow + e);
             if (static_cast<unsigned>(phys) >= static_cast<unsigned>(a.num_blocks)) {
               flag_error(a.err, PA_DEVERR_BLOCK_ID);
-              phys = 0;  // read a valid block instead; the result is flagged as wrong
+              phys = a.num_blocks;  // past the tensor map: TMA fills the tile with zeros
             }
           }
         }

@@ -188,6 +188,30 @@ def test_device_checks_flag_bad_inputs():
     assert pk.pa_device_error() == 0  # cleared by the previous read
 
 
+@pytest.mark.parametrize("variant", ["mma", "cuda_core"])
+@pytest.mark.parametrize("d,bs,schedule", [(128, 16, pk.PA_SCHEDULE_BALANCED), (128, 16, 64),
+                                           (64, 16, pk.PA_SCHEDULE_BALANCED), (64, 32, 0)])
+def test_bad_block_ids_read_zeros(variant, d, bs, schedule):
+    """A table entry outside [0, num_blocks) -- past the end or negative --
+    reads a block of zeros and flags PA_DEVERR_BLOCK_ID: the output equals the
+    oracle's over a pool whose extra block is all zeros."""
+    lens = [40, 100, 70]
+    q, pool, (t_ref, l_ref), (t, l) = make_case(lens, 8, 2, d, bs, seed=17 + d + bs)
+    nb = pool.shape[0]
+    bad = t.copy()
+    bad[0, 1] = nb + 5
+    bad[1, 0] = -3
+    bad[2, (70 - 1) // bs] = nb  # the ragged last block
+    zero_pool = torch.cat([pool, torch.zeros((1,) + tuple(pool.shape[1:]), dtype=pool.dtype)])
+    t_zero = t_ref.copy()
+    t_zero[0, 1] = t_zero[1, 0] = t_zero[2, (70 - 1) // bs] = nb
+    want = opa.decode(bf16_to_f64(q), bf16_to_f64(zero_pool), t_zero, l_ref, default_scale(d))
+    pk.pa_device_error(clear=True)
+    out = run_decode(q.cuda(), pool.cuda(), bad, l, default_scale(d), VARIANTS[variant], schedule)
+    assert pk.pa_device_error() == pk.PA_DEVERR_BLOCK_ID
+    compare(bf16_to_f64(out), want)
+
+
 def test_wait_timeout_is_reported():
     pk.pa_device_error(clear=True)
     pk.pa_selftest_wait_timeout(20_000_000)  # 20 ms

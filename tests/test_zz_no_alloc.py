@@ -7,8 +7,10 @@ synchronisation.  pa_decode_noalloc keeps the split-K partials in a fixed
 array compiled into the library instead.  These tests call it through the C
 ABI and check it against pa_decode (caller workspace) on two calls in a row,
 with inputs that need several sequence partitions, so the second call runs
-over scratch the first one left behind.  The file is named to be collected
-last; it passes alone in a fresh process as well.
+over scratch the first one left behind.  Both entry points run the same plan
+and kernels on the same inputs, so their outputs must be identical bit for
+bit; each is also checked against the fp64 oracle.  The file is named to be
+collected last; it passes alone in a fresh process as well.
 """
 
 import ctypes
@@ -19,8 +21,8 @@ import torch
 
 import paged_kv_cache_354_b200 as pk
 import workloads
-from tests.gpu_helpers import (MAX_ABS, MEAN_ABS, build_tables, poison_unused, run_decode,
-                               workspace_for)
+from oracle import paged_attention as opa
+from tests.gpu_helpers import bf16_to_f64, build_tables, compare, poison_unused, run_decode
 
 pytestmark = pytest.mark.gpu
 
@@ -30,10 +32,11 @@ HQ, HKV, D, BS = 16, 4, 128, 16
 def make_inputs(seed, lens):
     nb = sum(-(-int(n) // BS) for n in lens) + 8
     order = np.random.default_rng(seed).permutation(nb)
-    _, _, tables, lens32, used = build_tables(lens, BS, nb, order)
-    pool = poison_unused(workloads.bf16_normal((nb, 2, HKV, BS, D), seed=seed), used).cuda()
-    q = workloads.bf16_normal((len(lens), HQ, D), seed=seed + 1).cuda()
-    return q, pool, tables, lens32
+    t_ref, l_ref, tables, lens32, used = build_tables(lens, BS, nb, order)
+    pool = poison_unused(workloads.bf16_normal((nb, 2, HKV, BS, D), seed=seed), used)
+    q = workloads.bf16_normal((len(lens), HQ, D), seed=seed + 1)
+    want = opa.decode(bf16_to_f64(q), bf16_to_f64(pool), t_ref, l_ref, 1.0 / np.sqrt(D))
+    return q.cuda(), pool.cuda(), tables, lens32, want
 
 
 def call_noalloc(q, pool, tables, lens, max_len, scale):
@@ -57,17 +60,17 @@ def test_noalloc_matches_pa_decode_on_two_calls(seeds):
         (seeds[1], [1500, 2500, 33, 2047, 900, 16, 1024, 2900]),
     ]
     for seed, lens in cases:
-        q, pool, tables, lens32 = make_inputs(seed, lens)
+        q, pool, tables, lens32, oracle_out = make_inputs(seed, lens)
         max_len = max(lens)
         nbytes, parts = pk.pa_decode_workspace_size(len(lens), HQ, HKV, D, BS, max_len)
         assert parts > 1, "the case must use split-K scratch"
         assert 0 < nbytes <= pk.PA_NOALLOC_SCRATCH_BYTES
         scale = 1.0 / np.sqrt(D)
-        want = run_decode(q, pool, tables, lens32, scale).float()
-        got = call_noalloc(q, pool, tables, lens32, max_len, scale).float()
-        err = (got - want).abs()
+        want = run_decode(q, pool, tables, lens32, scale)
+        got = call_noalloc(q, pool, tables, lens32, max_len, scale)
         assert torch.isfinite(got).all()
-        assert err.max().item() <= MAX_ABS and err.mean().item() <= MEAN_ABS
+        assert torch.equal(got.view(torch.int16), want.view(torch.int16)), "differs from pa_decode"
+        compare(bf16_to_f64(got), oracle_out)
         assert pk.pa_device_error() == 0
 
 
