@@ -813,11 +813,11 @@ def study_multi_token(iters=30):
     assert pk.pa_device_error() == 0
 
 
-def study_variants(iters=20):
-    """Tensor-core vs CUDA-core consumer across GQA group sizes: pa_decode on
-    the llama8b lengths and shuffled pool, Hkv in {8, 32}, head dim 128 and
-    (Hkv 8) 64, groups 1, 2, 4, 8, 16, 32 (CUDA cores: 1, 2, 4); CUDA events
-    over back-to-back launches."""
+def study_variants(iters=20, hkvs=None, groups=None, only=None):
+    """The three consumers across GQA group sizes: pa_decode on the llama8b
+    lengths and shuffled pool, Hkv in {8, 32}, head dim 128 and (Hkv 8) 64,
+    groups 1, 2, 4, 8, 16, 32 -- mma.sync and tcgen05 for every group, CUDA
+    cores for 1, 2, 4; CUDA events over back-to-back launches."""
     import torch
 
     import paged_kv_cache_354_b200 as pk
@@ -828,6 +828,8 @@ def study_variants(iters=20):
     gen.manual_seed(workloads.seed_of("llama8b"))
     ws = torch.empty(64 << 20, dtype=torch.uint8, device=dev)
     for hkv, d in ((8, 128), (32, 128), (8, 64)):
+        if hkvs and (hkv, d) not in hkvs:
+            continue
         bs = 16
         pool = torch.randn((p.num_blocks, 2, hkv, bs, d), generator=gen, device=dev).bfloat16()
         alloc = pk.PaAlloc(p.num_blocks, bs, p.initial_order)
@@ -835,12 +837,15 @@ def study_variants(iters=20):
         tables, lens = alloc.block_tables(ids, -(-int(max(p.seq_lens)) // bs))
         d_t, d_l = torch.as_tensor(tables, device=dev), torch.as_tensor(lens, device=dev)
         for g in (1, 2, 4, 8, 16, 32):
+            if groups and g not in groups:
+                continue
             q = torch.randn((len(ids), hkv * g, d), generator=gen, device=dev).bfloat16()
             out = torch.empty_like(q)
             nbytes = decode_bytes(lens, hkv * g, hkv, d, bs)[0]
             res = {}
-            for name, variant in (("mma", pk.PA_DECODE_MMA), ("cuda_core", pk.PA_DECODE_CUDA_CORE)):
-                if variant == pk.PA_DECODE_CUDA_CORE and g not in (1, 2, 4):
+            for name, variant in (("mma", pk.PA_DECODE_MMA), ("cuda_core", pk.PA_DECODE_CUDA_CORE),
+                                  ("tcgen05", pk.PA_DECODE_TCGEN05)):
+                if (variant == pk.PA_DECODE_CUDA_CORE and g not in (1, 2, 4)) or (only and name != only):
                     continue
 
                 def call():
@@ -901,6 +906,14 @@ def main():
                     help="print the study's JSON lines instead of the benchmark line")
     ap.add_argument("--study-workload", choices=["llama8b", "mixed", "long"], default=None,
                     help="page-table study: one workload only (default: all three)")
+    ap.add_argument("--study-hkv", type=int, choices=[8, 32], default=None,
+                    help="variants study: one KV-head count only (with --study-head-dim)")
+    ap.add_argument("--study-head-dim", type=int, choices=[64, 128], default=128)
+    ap.add_argument("--study-group", type=int, choices=[1, 2, 4, 8, 16, 32], default=None,
+                    help="variants study: one GQA group only")
+    ap.add_argument("--study-variant", choices=["mma", "cuda_core", "tcgen05"], default=None,
+                    help="variants study: one consumer only")
+    ap.add_argument("--study-iters", type=int, default=None, help="timed launches per study point")
     ap.add_argument("--partition-tokens", type=int, default=0,
                     help="0 = library's choice; -1 = balanced schedule; N > 0 = per-partition grid of "
                          "N-token partitions")
@@ -922,7 +935,9 @@ def main():
     elif args.study == "read-bandwidth":
         study_read_bandwidth()
     elif args.study == "variants":
-        study_variants()
+        study_variants(iters=args.study_iters or 20,
+                       hkvs=[(args.study_hkv, args.study_head_dim)] if args.study_hkv else None,
+                       groups=[args.study_group] if args.study_group else None, only=args.study_variant)
     elif args.impl == "reference":
         run_reference(args)
     else:

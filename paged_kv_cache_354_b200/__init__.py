@@ -40,6 +40,7 @@ PA_DEVERR_COPY_PAIR = 0x10
 PA_DECODE_AUTO = 0
 PA_DECODE_CUDA_CORE = 1
 PA_DECODE_MMA = 2
+PA_DECODE_TCGEN05 = 3
 
 PA_SCHEDULE_BALANCED = -1  # partition_tokens value that asks for the balanced schedule
 

@@ -31,6 +31,7 @@
 
 #include <cmath>
 
+#include "pa_decode_common.cuh"
 #include "pa_device.cuh"
 #include "pa_internal.h"
 
@@ -42,7 +43,7 @@ constexpr int kMaxGroup = 8;
 constexpr float kRescaleSlack = 8.f;  // log2 units: probabilities stay <= 256
 constexpr unsigned kFull = 0xffffffffu;
 
-enum Variant { kCudaCore = 1, kMma = 2 };
+enum Variant { kCudaCore = 1, kMma = 2, kTc = 3 };
 
 template <int D, int BS>
 struct Geo {
@@ -75,46 +76,6 @@ struct Smem {
   static constexpr int kTotal = kFw + (kConsumerWarps * kMaxGroup + 2 * kMaxGroup) * 4;
   static constexpr int kDynamic = kTotal + 1024;                        // alignment slack
 };
-
-struct DecodeArgs {
-  __nv_bfloat16* out;
-  const __nv_bfloat16* q;
-  const int32_t* block_tables;
-  const int32_t* seq_lens;
-  float* part_o;  // [B*Hq][max_parts][D]
-  float* part_m;  // [B*Hq][max_parts]
-  float* part_l;  // [B*Hq][max_parts]
-  int32_t* err;
-  int num_q_heads, num_kv_heads, group;
-  int num_blocks, max_blocks_per_seq;
-  int len_cap;  // > 0: the longest length the table row holds (else max_blocks_per_seq * bs)
-  int part_blocks, max_parts;
-  float scale_log2;  // scale * log2(e)
-  int* stream_prefix;  // balanced schedule: per-request block-count prefix sums [B+1]
-  int qtok;            // query tokens per request (1 = single-token decode)
-  int cols;            // group * qtok: (token, head) columns per KV head
-  // fused cache write (pa_decode_append): request b's newest token, at
-  // position seq_lens[b] - 1, has keys/values new_k/new_v [B][Hkv][D] and
-  // slot new_slots[b] (< 0: nothing to write); null when not fused
-  const uint4* new_k;
-  const uint4* new_v;
-  const int64_t* new_slots;
-  uint4* pool_w;       // the pool, written by the merge kernel
-};
-
-// Tokens of request b the kernels attend over, after the device-side checks
-// (both kernels use this, so they agree on the partition count).
-__device__ __forceinline__ int effective_len(int raw, int bs, const DecodeArgs& a, bool report) {
-  int len = raw < 0 ? 0 : raw;
-  const int cap_table = a.len_cap > 0 ? a.len_cap : a.max_blocks_per_seq * bs;
-  const long long cap_grid = static_cast<long long>(a.max_parts) * a.part_blocks * bs;
-  if (len > cap_table || len > cap_grid || raw < 0) {
-    if (report) flag_error(a.err, PA_DEVERR_SEQ_LEN);
-    len = min(len, cap_table);
-    len = static_cast<int>(min(static_cast<long long>(len), cap_grid));
-  }
-  return len;
-}
 
 // --------------------------------------------------------------------------
 // Tensor-core consumer: state and per-block step.
@@ -799,96 +760,6 @@ struct StreamSmem {
   }
 };
 
-// First unit of the CTA range that contains unit u: the largest c with
-// floor(total * c / ctas) <= u.
-__device__ __forceinline__ long long stream_begin(long long total, int c, int ctas) {
-  return total * c / ctas;
-}
-__device__ __forceinline__ int stream_cta_of(long long total, long long u, int ctas) {
-  return static_cast<int>((static_cast<long long>(ctas) * (u + 1) + total - 1) / total - 1);
-}
-
-// (b, h, k) of unit u, from the block-count prefix sums (b with no blocks
-// are skipped because the largest b with hkv*prefix[b] <= u is taken).
-__device__ __forceinline__ void stream_locate(const int* prefix, int batch, int hkv, long long u,
-                                              int& b, int& h, int& k) {
-  int lo = 0, hi = batch - 1;
-  while (lo < hi) {
-    const int mid = (lo + hi + 1) >> 1;
-    if (static_cast<long long>(hkv) * prefix[mid] <= u) lo = mid;
-    else hi = mid - 1;
-  }
-  b = lo;
-  const int nb = prefix[b + 1] - prefix[b];
-  const long long r = u - static_cast<long long>(hkv) * prefix[b];
-  h = static_cast<int>(r / nb);
-  k = static_cast<int>(r - static_cast<long long>(h) * nb);
-}
-
-__device__ __forceinline__ void stream_next(const int* prefix, int batch, int hkv, int& b, int& h,
-                                            int& k) {
-  k = 0;
-  if (++h == hkv) {
-    h = 0;
-    do {
-      ++b;
-    } while (b < batch && prefix[b + 1] == prefix[b]);
-  }
-}
-
-// prefix[b] = sum_{b' < b} ceil(L_b' / bs) for b in [0, batch]; all threads.
-template <int BS>
-__device__ __forceinline__ void block_count_prefix(int* prefix, int* scan, int batch,
-                                                   const DecodeArgs& a, bool report) {
-  const int t = threadIdx.x;
-  const int per = (batch + kThreads - 1) / kThreads;
-  const int lo = min(batch, t * per);
-  const int hi = min(batch, lo + per);
-  int sum = 0;
-  for (int i = lo; i < hi; ++i) {
-    const int len = effective_len(__ldg(a.seq_lens + i), BS, a, report);
-    const int nb = (len + BS - 1) / BS;
-    prefix[i] = nb;
-    sum += nb;
-  }
-  scan[t] = sum;
-  __syncthreads();
-  if (t < 32) {  // exclusive scan of the kThreads partial sums by one warp
-    constexpr int kPer = (kThreads + 31) / 32;
-    int v[kPer];
-    int run = 0;
-#pragma unroll
-    for (int e = 0; e < kPer; ++e) {
-      const int idx = t * kPer + e;
-      v[e] = idx < kThreads ? scan[idx] : 0;
-      run += v[e];
-    }
-    int incl = run;
-#pragma unroll
-    for (int off = 1; off < 32; off <<= 1) {
-      const int y = __shfl_up_sync(kFull, incl, off);
-      if (t >= off) incl += y;
-    }
-    int excl = incl - run;
-#pragma unroll
-    for (int e = 0; e < kPer; ++e) {
-      const int idx = t * kPer + e;
-      if (idx < kThreads) scan[idx] = excl;
-      excl += v[e];
-    }
-    if (t == 31) scan[kThreads] = incl;  // grand total
-  }
-  __syncthreads();
-  int run = scan[t];
-  for (int i = lo; i < hi; ++i) {
-    const int nb = prefix[i];
-    prefix[i] = run;
-    run += nb;
-  }
-  if (t == 0) prefix[batch] = scan[kThreads];
-  __syncthreads();
-}
-
 __device__ __forceinline__ void consumer_bar() {
   asm volatile("bar.sync 1, %0;" ::"n"(kConsumerWarps * 32) : "memory");
 }
@@ -936,7 +807,7 @@ __global__ void __launch_bounds__(kThreads, kStreamCtasPerSm)
   }
   pdl_trigger();
   pdl_wait();  // every global access below comes after the previous grid
-  block_count_prefix<BS>(prefix, reinterpret_cast<int*>(smem + sm::kScan), batch, a,
+  block_count_prefix<BS, kThreads>(prefix, reinterpret_cast<int*>(smem + sm::kScan), batch, a,
                          blockIdx.x == 0);
   if (blockIdx.x == 0)
     for (int i = threadIdx.x; i <= batch; i += kThreads) a.stream_prefix[i] = prefix[i];
@@ -1211,7 +1082,8 @@ __global__ void __launch_bounds__(128) paged_decode_stream_merge_kernel(const De
   }
   const int* prefix = a.stream_prefix;
   const int pb0 = prefix[b], pb1 = prefix[b + 1], pall = prefix[batch];
-  const int nb = pb1 - pb0;
+  const int nbu = pb1 - pb0;                          // work units of each (b, h)
+  const int nb = nbu > 0 ? nbu - a.seg_extra : 0;     // of which real blocks
   __nv_bfloat16* o = a.out + static_cast<size_t>(gw) * D + lane * kPer;
   if (nb == 0) {
 #pragma unroll
@@ -1220,7 +1092,7 @@ __global__ void __launch_bounds__(128) paged_decode_stream_merge_kernel(const De
     return;
   }
   const long long total = static_cast<long long>(hkv) * pall;
-  const long long us = static_cast<long long>(hkv) * pb0 + static_cast<long long>(h) * nb;
+  const long long us = static_cast<long long>(hkv) * pb0 + static_cast<long long>(h) * nbu;
   const int c0 = stream_cta_of(total, us, ctas);
   const int c1 = stream_cta_of(total, us + nb - 1, ctas);
   if (c0 == c1) return;  // one CTA held the whole (b, h) and wrote the output
@@ -1493,6 +1365,18 @@ static int launch_stream(const CUtensorMap& map, const DecodeArgs& a, int batch,
   return PA_OK;
 }
 
+int launch_stream_merge(int d, int bs, const DecodeArgs& a, int batch, int ctas, cudaStream_t st) {
+  const int warps = batch * a.qtok * a.num_q_heads;
+  const dim3 grid((warps + 3) / 4);
+  cudaError_t e;
+  if (d == 64) e = bs == 16 ? launch_pdl(paged_decode_stream_merge_kernel<64, 16>, grid, dim3(128), 0, st, a, batch, ctas)
+                            : launch_pdl(paged_decode_stream_merge_kernel<64, 32>, grid, dim3(128), 0, st, a, batch, ctas);
+  else e = bs == 16 ? launch_pdl(paged_decode_stream_merge_kernel<128, 16>, grid, dim3(128), 0, st, a, batch, ctas)
+                    : launch_pdl(paged_decode_stream_merge_kernel<128, 32>, grid, dim3(128), 0, st, a, batch, ctas);
+  if (e != cudaSuccess) return fail(PA_ERR_CUDA, "merge launch: %s", cudaGetErrorString(e));
+  return PA_OK;
+}
+
 template <int D, int BS>
 static int dispatch(const CUtensorMap& map, const DecodeArgs& a, int batch, int variant,
                     const Plan& plan, cudaStream_t st) {
@@ -1579,14 +1463,23 @@ static int decode_impl(pa_bf16* out, const pa_bf16* q, const pa_bf16* kv_pool,
     return fail(PA_ERR_UNSUPPORTED, "group %d x query tokens %d above %d columns", group, qtok,
                 4 * kMaxGroup);
   if (qtok > 1 && variant == kCudaCore)
-    return fail(PA_ERR_UNSUPPORTED, "multi-token decode has the tensor-core variant only");
-  // tensor cores for every group: at scale they beat the CUDA-core consumer
-  // even where the group leaves most of the 8-wide tile empty (g = 1, 2)
-  if (variant == PA_DECODE_AUTO) variant = kMma;
+    return fail(PA_ERR_UNSUPPORTED, "multi-token decode has the tensor-core variants only");
+  // tensor cores for every group: at scale mma.sync beats the CUDA-core
+  // consumer even where the group leaves most of the 8-wide tile empty
+  // (g = 1, 2); from 9 to 16 columns the tcgen05 consumer takes over
+  if (variant == PA_DECODE_AUTO)
+    variant = (group * qtok > kMaxGroup && tc_decode_supported(d, bs, group * qtok)) ? kTc : kMma;
   if (variant == kCudaCore && group != 1 && group != 2 && group != 4)
     return fail(PA_ERR_UNSUPPORTED, "pa_decode: CUDA-core variant has no group size %d", group);
-  if (variant != kCudaCore && variant != kMma)
+  if (variant != kCudaCore && variant != kMma && variant != kTc)
     return fail(PA_ERR_INVALID, "pa_decode: unknown variant %d", variant);
+  if (variant == kTc) {  // the tcgen05 consumer exists on the balanced schedule only
+    if (!tc_decode_supported(d, bs, group * qtok))
+      return fail(PA_ERR_UNSUPPORTED, "pa_decode: the tcgen05 variant takes 1..16 columns, not %d", group * qtok);
+    if (partition_tokens > 0)
+      return fail(PA_ERR_UNSUPPORTED, "pa_decode: the tcgen05 variant runs on the balanced schedule only");
+    partition_tokens = kForceBalanced;
+  }
 
   Plan plan;
   rc = make_plan(batch, hq, hkv, d, bs, max_seq_len, partition_tokens, &plan, qtok);
@@ -1600,19 +1493,23 @@ static int decode_impl(pa_bf16* out, const pa_bf16* q, const pa_bf16* kv_pool,
   }
   int32_t* err = device_error_word();
   if (err == nullptr) return PA_ERR_CUDA;
-  const bool pairs = plan.stream && stream_tile(d, bs) != bs;
+  const bool tc = variant == kTc;
+  const bool pairs = !tc && plan.stream && stream_tile(d, bs) != bs;
 
   // TMA view of the pool: x = head dim, y = (kv head, row) of one K or V
   // plane of a block, z = 2*block + (0 keys | 1 values); a box brings both
   // planes, or (block pairs) one plane at a time.
+  // (the tcgen05 consumer encodes views of its own)
   alignas(64) CUtensorMap map;
-  const uint64_t dims[3] = {static_cast<uint64_t>(d), static_cast<uint64_t>(hkv) * bs,
-                            2ull * static_cast<uint64_t>(num_blocks)};
-  const uint64_t strides[2] = {static_cast<uint64_t>(d) * 2,
-                               static_cast<uint64_t>(hkv) * bs * d * 2};
-  const uint32_t box[3] = {64u, static_cast<uint32_t>(bs), pairs ? 1u : 2u};
-  rc = encode_tensor_map(&map, 3, const_cast<pa_bf16*>(kv_pool), dims, strides, box, 1);
-  if (rc != PA_OK) return rc;
+  if (!tc) {
+    const uint64_t dims[3] = {static_cast<uint64_t>(d), static_cast<uint64_t>(hkv) * bs,
+                              2ull * static_cast<uint64_t>(num_blocks)};
+    const uint64_t strides[2] = {static_cast<uint64_t>(d) * 2,
+                                 static_cast<uint64_t>(hkv) * bs * d * 2};
+    const uint32_t box[3] = {64u, static_cast<uint32_t>(bs), pairs ? 1u : 2u};
+    rc = encode_tensor_map(&map, 3, const_cast<pa_bf16*>(kv_pool), dims, strides, box, 1);
+    if (rc != PA_OK) return rc;
+  }
 
   DecodeArgs a;
   a.out = reinterpret_cast<__nv_bfloat16*>(out);
@@ -1640,11 +1537,13 @@ static int decode_impl(pa_bf16* out, const pa_bf16* q, const pa_bf16* kv_pool,
   a.new_v = nullptr;
   a.new_slots = nullptr;
   a.pool_w = reinterpret_cast<uint4*>(const_cast<pa_bf16*>(kv_pool));
+  a.seg_extra = tc ? tc_decode_segment_extra(bs) : 0;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   if (fused) {
     // the decode kernel patches the staged tile, the merge kernel stores the
-    // row; with block pairs or paired warps the cache write runs first
-    if (plan.stream && !pairs && a.cols <= kMaxGroup) {
+    // row; with block pairs, paired warps or the tcgen05 consumer the cache
+    // write runs first
+    if (plan.stream && !pairs && !tc && a.cols <= kMaxGroup) {
       a.new_k = reinterpret_cast<const uint4*>(new_k);
       a.new_v = reinterpret_cast<const uint4*>(new_v);
       a.new_slots = new_slots;
@@ -1655,6 +1554,7 @@ static int decode_impl(pa_bf16* out, const pa_bf16* q, const pa_bf16* kv_pool,
     }
   }
 
+  if (tc) return launch_tc_decode(a, kv_pool, batch, d, bs, num_blocks, sm_count() > 0 ? sm_count() : 148, st);
   if (pairs) return dispatch_pairs(map, a, batch, variant, plan.ctas, st);
   if (d == 64 && bs == 16) return dispatch<64, 16>(map, a, batch, variant, plan, st);
   if (d == 64 && bs == 32) return dispatch<64, 32>(map, a, batch, variant, plan, st);
@@ -1808,7 +1708,7 @@ int pa_decode_multi(pa_bf16* out, const pa_bf16* q, const pa_bf16* kv_pool,
                     float scale, void* workspace, size_t workspace_bytes, void* stream) {
   return pa::decode_impl(out, q, kv_pool, block_tables, seq_lens, batch, num_q_heads, num_kv_heads,
                          head_dim, block_size, num_blocks, max_blocks_per_seq, max_seq_len, scale,
-                         workspace, workspace_bytes, PA_DECODE_MMA, pa::kForceBalanced, stream,
+                         workspace, workspace_bytes, PA_DECODE_AUTO, pa::kForceBalanced, stream,
                          num_query_tokens);
 }
 

@@ -92,6 +92,21 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
   return done != 0;
 }
 
+// Non-blocking test of the same condition (try_wait may suspend the thread
+// for a while when the phase is not complete; a thread that polls several
+// barriers in turn needs the test that returns at once).
+__device__ __forceinline__ bool mbar_test_wait(uint32_t bar, uint32_t parity) {
+  uint32_t done;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(done)
+      : "r"(bar), "r"(parity)
+      : "memory");
+  return done != 0;
+}
+
 // Wait for the phase of parity `parity` to complete, for at most limit_ns.
 // Returns false when the limit ran out (the caller records the timeout and
 // unwinds; nothing here traps or spins forever).

@@ -77,7 +77,9 @@ def run_decode(q, pool, tables, lens, scale, variant=pk.PA_DECODE_AUTO, partitio
     b, hq, d = q.shape
     hkv, bs = pool.shape[2], pool.shape[3]
     max_len = int(max(1, int(lens.max()) if len(lens) else 1))
-    ws, _ = workspace_for(b, hq, hkv, d, bs, max_len, partition_tokens)
+    # the tcgen05 consumer always runs the balanced schedule: size for it
+    ws_schedule = pk.PA_SCHEDULE_BALANCED if variant == pk.PA_DECODE_TCGEN05 else partition_tokens
+    ws, _ = workspace_for(b, hq, hkv, d, bs, max_len, ws_schedule)
     out = torch.full_like(q, float("nan"))
     pk.pa_decode(out, q, pool, torch.as_tensor(tables, device="cuda"), torch.as_tensor(lens, device="cuda"),
                  max_len, scale, workspace=ws, variant=variant, partition_tokens=partition_tokens)

@@ -18,7 +18,8 @@ import workloads
 
 pytestmark = pytest.mark.gpu
 
-VARIANTS = {"auto": pk.PA_DECODE_AUTO, "cuda_core": pk.PA_DECODE_CUDA_CORE, "mma": pk.PA_DECODE_MMA}
+VARIANTS = {"auto": pk.PA_DECODE_AUTO, "cuda_core": pk.PA_DECODE_CUDA_CORE, "mma": pk.PA_DECODE_MMA,
+            "tcgen05": pk.PA_DECODE_TCGEN05}
 
 
 def make_case(lens, hq, hkv, d, bs, seed, extra_blocks=4):
@@ -77,10 +78,11 @@ def test_split_k_partitions(partition_blocks, variant):
     [40000],                   # one request cut across every CTA
     [17, 40000, 0, 5, 2048],   # mixed, with a request split many ways
 ])
-@pytest.mark.parametrize("variant", ["mma", "cuda_core"])
+@pytest.mark.parametrize("variant", ["mma", "cuda_core", "tcgen05"])
 def test_balanced_schedule_edges(lens, variant):
-    check(lens, 8 if variant == "mma" else 4, 2 if variant == "mma" else 4, 64, 16, seed=60 + len(lens),
-          variant=variant, partition_tokens=pk.PA_SCHEDULE_BALANCED)
+    hq, hkv = {"mma": (8, 2), "cuda_core": (4, 4), "tcgen05": (32, 2)}[variant]
+    for d in (64, 128) if variant == "tcgen05" else (64,):
+        check(lens, hq, hkv, d, 16, seed=60 + len(lens), variant=variant, partition_tokens=pk.PA_SCHEDULE_BALANCED)
 
 
 def test_balanced_matches_partition_grid():
@@ -95,10 +97,39 @@ def test_balanced_matches_partition_grid():
 @pytest.mark.parametrize("d,bs", [(128, 16), (64, 32), (64, 16)])
 @pytest.mark.parametrize("schedule", [0, pk.PA_SCHEDULE_BALANCED])
 @pytest.mark.parametrize("hq,hkv", [(32, 2), (24, 2), (64, 2), (32, 1)])
-def test_wide_groups(d, bs, schedule, hq, hkv):
-    """Groups of 12, 16 and 32 query heads per KV head (32/1: multi-query):
-    two or four 8-wide MMA tiles on grouped warps (balanced schedule only)."""
-    check(RAGGED, hq, hkv, d, bs, seed=70 + d + bs + hq, partition_tokens=schedule)
+@pytest.mark.parametrize("variant", ["auto", "mma"])
+def test_wide_groups(d, bs, schedule, hq, hkv, variant):
+    """Groups of 12, 16 and 32 query heads per KV head (32/1: multi-query),
+    balanced schedule only: by default the tcgen05 consumer; on request
+    mma.sync with two or four 8-wide MMA tiles on grouped warps."""
+    check(RAGGED, hq, hkv, d, bs, seed=70 + d + bs + hq, variant=variant, partition_tokens=schedule)
+
+
+@pytest.mark.parametrize("d,bs", [(128, 16), (128, 32), (64, 16), (64, 32)])
+@pytest.mark.parametrize("hq,hkv", [(2, 2), (8, 2), (18, 2), (26, 2), (32, 2), (16, 1), (96, 8)])
+def test_tcgen05_variant(d, bs, hq, hkv):
+    """The tcgen05 consumer for 1..16 (token, head) columns (one 16-column
+    MMA tile): 128-token tiles with ragged ends, tiles cut between CTAs,
+    requests of exactly one tile, NaN in every unused pool row."""
+    check(RAGGED + [2000, 129, 128, 127, 4111], hq, hkv, d, bs, seed=300 + d + bs + hq + hkv, variant="tcgen05")
+
+
+def test_tcgen05_rejects_more_than_16_columns():
+    q, pool, _, (t, l) = make_case([40, 70], 34, 2, 128, 16, seed=301)
+    with pytest.raises(pk.PaError):
+        run_decode(q.cuda(), pool.cuda(), t, l, 0.1, pk.PA_DECODE_TCGEN05)
+
+
+@pytest.mark.parametrize("hq,hkv", [(24, 2), (32, 2)])
+def test_tcgen05_matches_mma_sync(hq, hkv):
+    """Both tensor-core consumers on the same wide-group inputs: equal up to
+    the rounding of their different summation orders."""
+    lens = [3000, 17, 1200, 2049, 5, 640, 2999, 1, 4096, 33]
+    q, pool, _, (t, l) = make_case(lens, hq, hkv, 128, 16, seed=64 + hq)
+    q, pool = q.cuda(), pool.cuda()
+    a = run_decode(q, pool, t, l, 0.088, pk.PA_DECODE_TCGEN05)
+    b = run_decode(q, pool, t, l, 0.088, pk.PA_DECODE_MMA, partition_tokens=pk.PA_SCHEDULE_BALANCED)
+    assert (a.float() - b.float()).abs().max().item() <= 2 ** -7
 
 
 def test_balanced_schedule_at_its_batch_limit():
@@ -154,9 +185,13 @@ def test_zero_length_request():
 
 
 def test_large_logits():
-    """A large scale makes the softmax nearly one-hot; the online max must hold."""
+    """A large scale makes the softmax nearly one-hot; the online max must hold
+    (for the wide groups: the column maxima and the rescale of O in tensor
+    memory)."""
     check([77, 500], 8, 2, 128, 16, seed=13, scale=4.0)
     check([77, 500], 4, 4, 64, 16, seed=14, scale=4.0)
+    check([77, 500, 3000], 32, 2, 128, 16, seed=15, scale=4.0, variant="tcgen05")
+    check([77, 500, 3000], 24, 2, 64, 32, seed=16, scale=4.0, variant="tcgen05")
 
 
 def test_tiny_workload():
@@ -188,9 +223,13 @@ def test_device_checks_flag_bad_inputs():
     assert pk.pa_device_error() == 0  # cleared by the previous read
 
 
-@pytest.mark.parametrize("variant", ["mma", "cuda_core"])
-@pytest.mark.parametrize("d,bs,schedule", [(128, 16, pk.PA_SCHEDULE_BALANCED), (128, 16, 64),
-                                           (64, 16, pk.PA_SCHEDULE_BALANCED), (64, 32, 0)])
+BAD_ID_CASES = [(v, 128, 16, pk.PA_SCHEDULE_BALANCED) for v in ("mma", "cuda_core", "tcgen05")] + \
+    [(v, 128, 16, 64) for v in ("mma", "cuda_core")] + \
+    [(v, 64, 16, pk.PA_SCHEDULE_BALANCED) for v in ("mma", "cuda_core", "tcgen05")] + \
+    [(v, 64, 32, 0) for v in ("mma", "cuda_core", "tcgen05")]
+
+
+@pytest.mark.parametrize("variant,d,bs,schedule", BAD_ID_CASES)
 def test_bad_block_ids_read_zeros(variant, d, bs, schedule):
     """A table entry outside [0, num_blocks) -- past the end or negative --
     reads a block of zeros and flags PA_DEVERR_BLOCK_ID: the output equals the

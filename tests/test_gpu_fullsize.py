@@ -145,3 +145,31 @@ def test_full_size_multi_token_whole_batch():
     t_ref, l_ref = workloads.block_tables(ref, ids_r)
     want = oracle_batch_multi(q.double().cpu().numpy(), pool_u16, t_ref, l_ref, s.block_size, scale)
     assert_close(out.double().cpu().numpy(), want)
+
+
+@pytest.mark.parametrize("group", [16, 32])
+def test_full_size_wide_group_whole_batch(group):
+    """The Llama-3-8B decode workload's lengths, pool and tables with 16 or 32
+    query heads per KV head (the tcgen05 consumer): every output against the
+    oracle."""
+    dev = torch.device("cuda", torch.cuda.current_device())
+    p, cache, ids, gen = bench.build_cache("llama8b", 2, 0, dev, prefill=False)
+    s = p.shape
+    hq = s.num_kv_heads * group
+    pool_u16 = bits(cache.pool)
+    tables, lens = cache.alloc.block_tables(ids, cache.max_blocks)
+    q = torch.randn((len(ids), hq, s.head_dim), generator=gen, device=dev).bfloat16()
+    out = torch.full_like(q, float("nan"))
+    scale = 1.0 / math.sqrt(s.head_dim)
+    nbytes, _ = pk.pa_decode_workspace_size(len(ids), hq, s.num_kv_heads, s.head_dim, s.block_size,
+                                            cache.max_seq_len)
+    ws = torch.empty(max(256, nbytes), dtype=torch.uint8, device=dev)
+    pk.pa_device_error(clear=True)
+    pk.pa_decode(out, q, cache.pool, torch.as_tensor(tables, device=dev), torch.as_tensor(lens, device=dev),
+                 cache.max_seq_len, scale, workspace=ws)
+    torch.cuda.synchronize()
+    assert pk.pa_device_error() == 0
+    ref = BlockAllocator(p.num_blocks, s.block_size, p.initial_order)
+    t_ref, l_ref = workloads.block_tables(ref, workloads.populate(ref, p))
+    want = oracle_batch(q.double().cpu().numpy(), pool_u16, t_ref, l_ref, s.block_size, scale)
+    assert_close(out.double().cpu().numpy(), want)
