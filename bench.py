@@ -43,7 +43,9 @@ SPEC_HBM_GBS = 8000.0  # B200 data-sheet HBM3e bandwidth
 
 
 TRAFFIC_FILE = os.path.join(ROOT, "profiles", "paged_decode_traffic.json")
-DECODE_SOURCES = ("paged_kv_cache_354_b200/csrc/pa_decode.cu", "paged_kv_cache_354_b200/csrc/pa_device.cuh")
+DECODE_SOURCES = ("paged_kv_cache_354_b200/csrc/pa_decode.cu", "paged_kv_cache_354_b200/csrc/pa_device.cuh",
+                  "paged_kv_cache_354_b200/csrc/pa_decode_common.cuh", "paged_kv_cache_354_b200/csrc/pa_decode_tc.cu",
+                  "paged_kv_cache_354_b200/csrc/pa_tcgen05.cuh")
 
 
 def decode_source_digest():

@@ -710,6 +710,14 @@ __global__ void __launch_bounds__(kThreads, (VAR == kMma || G <= 2) ? 3 : 2)
 #define PA_STREAM_RING_BYTES 65536
 #endif
 constexpr int kStreamCtasPerSm = PA_STREAM_CTAS_PER_SM;
+// Per-segment cost of the balanced kernel (segment epilogue, a pipeline
+// drain at the segment's end) in tokens' worth of streaming: the split
+// counts this many virtual tokens for every (request, KV head) so the CTAs
+// covering many short requests finish with the others.
+#ifndef PA_STREAM_SEG_EXTRA_TOKENS
+#define PA_STREAM_SEG_EXTRA_TOKENS 64
+#endif
+constexpr int kStreamSegExtraTokens = PA_STREAM_SEG_EXTRA_TOKENS;
 constexpr int kStreamMaxBatch = 4096;  // the prefix table lives in shared memory
 
 // Consumer groups of the balanced kernel: with up to 8 (token, head) columns
@@ -827,8 +835,12 @@ __global__ void __launch_bounds__(kThreads, kStreamCtasPerSm)
     int i = 0;  // running block index in this CTA
     bool stop = false;
     while (u < u_end && !stop) {
-      const int nb = prefix[b + 1] - prefix[b];
-      const int cnt = static_cast<int>(min(static_cast<long long>(nb - k), u_end - u));
+      // the (b, h) spans nbu units: nb real tiles, then a.seg_extra virtual
+      // ones of the overhead-weighted split (no data, skipped)
+      const int nbu = prefix[b + 1] - prefix[b];
+      const int nb = nbu - a.seg_extra;
+      const int cnt_u = static_cast<int>(min(static_cast<long long>(nbu - k), u_end - u));
+      const int cnt = max(0, min(k + cnt_u, nb) - k);  // real tiles of this segment
       constexpr int kPerFetch = LAYOUT == kPagedPairs ? 16 : 32;  // tiles per table fetch
       // physical blocks of request b (the pair layout's last tile may hold one)
       const int nphys = LAYOUT == kPagedPairs
@@ -899,7 +911,7 @@ __global__ void __launch_bounds__(kThreads, kStreamCtasPerSm)
         }
       }
       i += cnt;
-      u += cnt;
+      u += cnt_u;
       stream_next(prefix, batch, hkv, b, h, k);
     }
   } else {
@@ -919,8 +931,11 @@ __global__ void __launch_bounds__(kThreads, kStreamCtasPerSm)
     int i = 0;
     int seg = 0;
     while (u < u_end) {
-      const int nb = prefix[b + 1] - prefix[b];
-      const int cnt = static_cast<int>(min(static_cast<long long>(nb - k), u_end - u));
+      const int nbu = prefix[b + 1] - prefix[b];  // units: nb real tiles + the split's virtual ones
+      const int nb = nbu - a.seg_extra;
+      const int cnt_u = static_cast<int>(min(static_cast<long long>(nbu - k), u_end - u));
+      const int cnt = max(0, min(k + cnt_u, nb) - k);  // real tiles of this segment
+      if (cnt > 0) {  // (uniform over the consumer warps: a virtual-only segment is skipped)
       const bool complete = (k == 0 && cnt == nb);
       // Q row of (token 0, head 0) of this KV head's group; out rows alike
       const size_t qrow0 = static_cast<size_t>(b) * a.qtok * a.num_q_heads + static_cast<size_t>(h) * g;
@@ -1024,8 +1039,9 @@ __global__ void __launch_bounds__(kThreads, kStreamCtasPerSm)
         }
       }
       consumer_bar();  // the scratch is free for the next segment
+      }  // cnt > 0
       i += cnt;
-      u += cnt;
+      u += cnt_u;
       ++seg;
       stream_next(prefix, batch, hkv, b, h, k);
     }
@@ -1537,7 +1553,9 @@ static int decode_impl(pa_bf16* out, const pa_bf16* q, const pa_bf16* kv_pool,
   a.new_v = nullptr;
   a.new_slots = nullptr;
   a.pool_w = reinterpret_cast<uint4*>(const_cast<pa_bf16*>(kv_pool));
-  a.seg_extra = tc ? tc_decode_segment_extra(bs) : 0;
+  // overhead-weighted split of the balanced schedule (virtual units per
+  // (request, KV head), in the kernel's tiles)
+  a.seg_extra = tc ? tc_decode_segment_extra(bs) : (plan.stream ? kStreamSegExtraTokens / stream_tile(d, bs) : 0);
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   if (fused) {
     // the decode kernel patches the staged tile, the merge kernel stores the
@@ -1655,6 +1673,9 @@ static int decode_contiguous_impl(pa_bf16* out, const pa_bf16* q, const pa_bf16*
   a.new_v = nullptr;
   a.new_slots = nullptr;
   a.pool_w = nullptr;
+  // the paged kernel's split, so that at equal lengths both layouts cut the
+  // same (request, head) pairs and merge them in the same order
+  a.seg_extra = kStreamSegExtraTokens / kContiguousTile;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   if (d == 64) return dispatch_contiguous<64>(map, a, batch, variant, plan.ctas, st);
   return dispatch_contiguous<128>(map, a, batch, variant, plan.ctas, st);
