@@ -308,7 +308,7 @@ def device_arm(name, K, W, rank, device, world, variant=0, partition_tokens=0, m
     import torch
     import torch.distributed as dist
 
-    p, cache, ids, gen = build_cache(name, 2 * (W + K) + 4, rank, device, variant=variant,
+    p, cache, ids, gen = build_cache(name, steps_total(W, K), rank, device, variant=variant,
                                      partition_tokens=partition_tokens)
     batch = len(ids)
     qs, ks, vs = make_inputs(cache, batch, gen, device)
@@ -355,13 +355,22 @@ def device_arm(name, K, W, rank, device, world, variant=0, partition_tokens=0, m
     }
 
 
+E2E_BLOCK = 10  # steps per block; blocks of the two output paths alternate
+
+
 def e2e_arm(arm, K, W, device, world):
-    """End to end through the engine, K steps: per step the host allocator
-    writes the step's metadata into a pinned staging buffer that already
-    holds the step's q/k/v; one CUDA graph copies it to the device, runs the
-    fused cache write + decode + merge and copies the output back; the
-    allocator work for step i+1 runs on the host while the GPU works on
-    step i; the host waits for step i's output before going on."""
+    """End to end through the engine, for both ways the output can reach
+    the host.  Per step the host allocator writes the step's metadata into a
+    pinned staging buffer that already holds the step's q/k/v; one CUDA
+    graph copies it to the device and runs the fused cache write + decode +
+    merge, whose kernels either store the output straight into pinned host
+    memory ("zero_copy") or write it on the device for a D2H copy at the end
+    of the graph ("copy"); the allocator work for step i+1 runs on the host
+    while the GPU works on step i; the host waits for step i's output before
+    going on.  One timed loop of 2K steps runs blocks of E2E_BLOCK steps of
+    each path in turn (so both see the same lengths), a CUDA event at every
+    block boundary; returns {path: (ms, bytes)} over its K steps and the H2D
+    and D2H bytes per step."""
     import torch
     import torch.distributed as dist
 
@@ -375,10 +384,10 @@ def e2e_arm(arm, K, W, device, world):
     e2e_lens = []
     pending = {}
 
-    def e2e_step(i):
+    def e2e_step(i, zero_copy):
         # step i's metadata was staged in buffer j during step i-1
         j = i % INPUT_SETS
-        cache.replay_step(j, pending.pop(i))  # upload, decode, output copy: one graph
+        cache.replay_step(j, pending.pop(i), zero_copy)  # upload, decode, output to the host: one graph
         e2e_lens.append(cache.staged("lens", j).numpy().copy())  # bookkeeping while the GPU works
         pending[i + 1] = cache.host_step(ids, (i + 1) % INPUT_SETS)
         stream.synchronize()  # the step's result is on the host
@@ -386,17 +395,44 @@ def e2e_arm(arm, K, W, device, world):
     cache.host_step(ids, 0)  # one eager step, then record the graphs on its staged data
     cache.upload(0)
     cache.capture(out)
-    cache.capture_steps(out, h_out)
+    cache.capture_steps(out, h_out, zero_copy=False)
+    cache.capture_steps(out, h_out, zero_copy=True)
     pending[0] = cache.host_step(ids, 0)
-    for i in range(W):
-        e2e_step(i)
+    for i in range(2 * W):
+        e2e_step(i, i % 2 == 0)
     torch.cuda.synchronize()
     if world > 1:
         dist.barrier()
+    blocks = []  # (path, first step, steps)
+    done = {"zero_copy": 0, "copy": 0}
+    while done["zero_copy"] < K or done["copy"] < K:
+        for path in ("zero_copy", "copy"):
+            n = min(E2E_BLOCK, K - done[path])
+            if n > 0:
+                blocks.append((path, 2 * W + done["zero_copy"] + done["copy"], n))
+                done[path] += n
+    events = [torch.cuda.Event(enable_timing=True) for _ in range(len(blocks) + 1)]
     e2e_lens.clear()
-    ms = timed_ms(stream, lambda: [e2e_step(W + i) for i in range(K)])
-    nbytes = sum(decode_bytes(ln, cache.hq, cache.hkv, cache.d, cache.bs)[0] for ln in e2e_lens)
-    return ms, nbytes, cache.stage_bytes, int(h_out.nbytes)
+    torch.cuda.synchronize()
+    for b, (path, first, n) in enumerate(blocks):
+        events[b].record(stream)
+        for i in range(first, first + n):
+            e2e_step(i, path == "zero_copy")
+    events[-1].record(stream)
+    torch.cuda.synchronize()
+    results = {"zero_copy": [0.0, 0], "copy": [0.0, 0]}
+    for b, (path, first, n) in enumerate(blocks):
+        results[path][0] += events[b].elapsed_time(events[b + 1])
+        lens_b = e2e_lens[first - 2 * W:first - 2 * W + n]
+        results[path][1] += sum(decode_bytes(ln, cache.hq, cache.hkv, cache.d, cache.bs)[0] for ln in lens_b)
+    return {k: tuple(v) for k, v in results.items()}, cache.stage_bytes, int(h_out.nbytes)
+
+
+def steps_total(W, K):
+    """Tokens each request may gain over a run (device arm, the e2e loop
+    over both output paths, slack): sizes the workload's pool, so both arms'
+    configs use it."""
+    return 3 * (W + K) + 8
 
 
 def workload_entry(name, arm, peaks, world):
@@ -440,13 +476,14 @@ def run_gpu(args):
     K, W = args.steps, args.warmup
     variant = {"auto": 0, "cuda_core": 1, "mma": 2}[args.variant]
     arm = device_arm(args.workload, K, W, rank, device, world, variant, args.partition_tokens, args.min_seconds)
-    e2e_ms, e2e_bytes, stage_bytes, d2h_bytes = e2e_arm(arm, K, W, device, world)
+    e2e, stage_bytes, d2h_bytes = e2e_arm(arm, K, W, device, world)
     dev_err = pa_device_error()
 
     # ---- max over ranks (times), sum over ranks (work)
-    step_ms, e2e_ms, decode_ms, bytes_all, e2e_bytes_all, kv_all = combine_ranks(
-        [arm["step_ms"], e2e_ms, arm["decode_ms"]], [arm["bytes_timed"], e2e_bytes, arm["kv_timed"]], device,
-        world)
+    (step_ms, e2e_ms, e2e_copy_ms, decode_ms, bytes_all, e2e_bytes_all, e2e_copy_bytes_all,
+     kv_all) = combine_ranks([arm["step_ms"], e2e["zero_copy"][0], e2e["copy"][0], arm["decode_ms"]],
+                             [arm["bytes_timed"], e2e["zero_copy"][1], e2e["copy"][1], arm["kv_timed"]],
+                             device, world)
     cache, steps_timed = arm["cache"], arm["steps_timed"]
     batch = len(arm["ids"])
     summary = {
@@ -490,7 +527,7 @@ def run_gpu(args):
             "vs_baseline": None,
             "dtype": "bf16",
             "data": "synthetic (seeded bf16 N(0,1) q/K/V; seeded lengths and shuffled block pool)",
-            "config": workload_config(args.workload, 2 * (W + K) + 4, world),
+            "config": workload_config(args.workload, steps_total(W, K), world),
             "run": {**summary, "timed_repeats": steps_timed // K, "steps_timed": steps_timed,
                     "timing": "the K steps repeated timed_repeats times back to back (each repetition the same "
                               "K steps: copy-on-write copies, fused cache write + decode + merge); one pair of "
@@ -521,9 +558,19 @@ def run_gpu(args):
                 "ms_per_step": round(e2e_ms / K, 5),
                 "steps_timed": K,
                 "path": "per step: one CUDA graph holding the H2D copy of a pinned staging buffer "
-                        "(metadata from the C++ allocator + the step's q/k/v), the fused cache write + "
-                        "decode + merge and the D2H copy of the output; then a sync; the allocator work "
+                        "(metadata from the C++ allocator + the step's q/k/v) and the fused cache write + "
+                        "decode + merge, whose kernels store the output rows straight into pinned host "
+                        "memory across PCIe as they finish (zero-copy); then a sync; the allocator work "
                         "for the next step runs on the host while the GPU works",
+                "with_d2h_copy": {
+                    "value": round(e2e_copy_bytes_all / (e2e_copy_ms * 1e-3) / 1e9, 2),
+                    "ms_per_step": round(e2e_copy_ms / K, 5),
+                    "path": "the same steps with the output written on the device and one D2H copy "
+                            "of it at the end of the graph",
+                },
+                "timing": f"one loop of 2K steps, blocks of {E2E_BLOCK} steps of each output path in "
+                          "turn (equal lengths for both), CUDA events at the block boundaries; each "
+                          "path's ms_per_step = its blocks' time / K",
             },
             "gpu_launches": launches * world,  # the step loop (value's timed region), every rank
             "clocks": clocks,
@@ -631,7 +678,7 @@ def run_reference(args):
         "vs_baseline": None,
         "dtype": "f64",
         "data": "synthetic (seeded bf16 N(0,1) K/V and q, upcast to f64)",
-        "config": workload_config(args.workload, 2 * (args.warmup + args.steps) + 4,
+        "config": workload_config(args.workload, steps_total(args.warmup, args.steps),
                                   int(os.environ.get("WORLD_SIZE", "1"))),
         "run": {"note": "each step decodes at least one whole request of the workload on the host"},
         "cpu_baseline": {"value": round(value, 4), "unit": "GB/s", "cores": 1, "kind": "oracle",

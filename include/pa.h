@@ -136,7 +136,14 @@ int pa_copy_blocks(pa_bf16* kv_pool, const int32_t* block_pairs, int num_pairs,
  * the P.V product); out is rounded to bf16 (round-to-nearest-even).
  * A request with seq_len 0 gets out = 0.
  *
- * out          : device bf16 [batch][num_q_heads][head_dim]
+ * out          : bf16 [batch][num_q_heads][head_dim], in device memory or
+ *                in page-locked host memory that the device addresses at
+ *                the same pointer (cudaHostAlloc, or cudaHostRegister,
+ *                under unified addressing).  In host memory the kernels
+ *                store each output row across PCIe as it becomes final
+ *                (zero-copy): it is complete once the stream has passed
+ *                the call.  Pageable or unknown memory: PA_ERR_INVALID
+ *                before any launch.  Only written, never read.
  * q            : device bf16 [batch][num_q_heads][head_dim]
  * kv_pool      : device bf16 pool (layout above); rows beyond a request's
  *                length inside its last block may hold anything (even NaN).
@@ -278,7 +285,9 @@ int pa_decode_append(pa_bf16* out, const pa_bf16* q, pa_bf16* kv_pool, const pa_
  * prefix.  A token with no position to attend to (seq_lens[b] < T - t) gets
  * out = 0.
  *
- * q, out       : device bf16 [batch][T][num_q_heads][head_dim]
+ * q, out       : bf16 [batch][T][num_q_heads][head_dim]; q in device
+ *                memory, out in device or pinned host memory as for
+ *                pa_decode
  * Other arguments as pa_decode.  (num_q_heads / num_kv_heads) * T <= 32.
  * Always the balanced schedule (batch <= 4096) and a tensor-core consumer
  * (tcgen05 for 9..16 columns, mma.sync otherwise); workspace from
@@ -315,7 +324,7 @@ int pa_decode_multi(pa_bf16* out, const pa_bf16* q, const pa_bf16* kv_pool,
  * PA_DECODE_CUDA_CORE (group 1, 2, 4) or PA_DECODE_MMA.  batch <= 4096,
  * group <= 8.
  * Workspace from pa_decode_contiguous_workspace_size (never 0 bytes).
- * Other arguments as pa_decode.
+ * Other arguments as pa_decode (out in device or pinned host memory).
  * ------------------------------------------------------------------------ */
 int pa_decode_contiguous_workspace_size(int batch, int num_q_heads, int num_kv_heads, int head_dim,
                                         int max_len, size_t* bytes_out);

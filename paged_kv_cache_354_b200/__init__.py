@@ -135,11 +135,11 @@ def _stream(stream):
     return ctypes.c_void_p(stream.cuda_stream)
 
 
-def _require(t, dtype, name):
+def _require(t, dtype, name, pinned_ok=False):
     if t.dtype != dtype:
         raise TypeError(f"{name}: expected {dtype}, got {t.dtype}")
-    if not t.is_cuda:
-        raise TypeError(f"{name}: expected a CUDA tensor")
+    if not t.is_cuda and not (pinned_ok and t.is_pinned()):
+        raise TypeError(f"{name}: expected a CUDA tensor" + (" or a pinned host tensor" if pinned_ok else ""))
     if not t.is_contiguous():
         raise ValueError(f"{name}: expected a contiguous tensor")
 
@@ -204,10 +204,12 @@ def pa_decode_workspace_size(batch, num_q_heads, num_kv_heads, head_dim, block_s
 
 def pa_decode(out, q, kv_pool, block_tables, seq_lens, max_seq_len, scale, workspace=None,
               variant=PA_DECODE_AUTO, partition_tokens=0, stream=None):
-    """Paged decode attention; writes ``out`` (bf16 [B, Hq, D]) in place."""
+    """Paged decode attention; writes ``out`` (bf16 [B, Hq, D]) in place.
+    ``out`` is a CUDA tensor or a pinned host tensor (the kernels then store
+    the rows across PCIe as they finish; read it after the stream syncs)."""
     import torch
 
-    _require(out, torch.bfloat16, "out")
+    _require(out, torch.bfloat16, "out", pinned_ok=True)
     _require(q, torch.bfloat16, "q")
     _require(kv_pool, torch.bfloat16, "kv_pool")
     _require(block_tables, torch.int32, "block_tables")
@@ -238,7 +240,7 @@ def pa_decode_multi(out, q, kv_pool, block_tables, seq_lens, max_seq_len, scale,
     """T causal query tokens per request: q, out bf16 [B, T, Hq, D]."""
     import torch
 
-    _require(out, torch.bfloat16, "out")
+    _require(out, torch.bfloat16, "out", pinned_ok=True)
     _require(q, torch.bfloat16, "q")
     _require(kv_pool, torch.bfloat16, "kv_pool")
     _require(block_tables, torch.int32, "block_tables")
@@ -265,7 +267,7 @@ def pa_decode_contiguous(out, q, kv_cache, seq_lens, scale, workspace, variant=P
     [B, 2, Hkv, max_len, D] (no block table); writes ``out`` in place."""
     import torch
 
-    _require(out, torch.bfloat16, "out")
+    _require(out, torch.bfloat16, "out", pinned_ok=True)
     _require(q, torch.bfloat16, "q")
     _require(kv_cache, torch.bfloat16, "kv_cache")
     _require(seq_lens, torch.int32, "seq_lens")
@@ -289,7 +291,7 @@ def pa_decode_noalloc(out, q, kv_pool, block_tables, seq_lens, max_seq_len, scal
     device; calls that overlap on the GPU race on it)."""
     import torch
 
-    _require(out, torch.bfloat16, "out")
+    _require(out, torch.bfloat16, "out", pinned_ok=True)
     _require(q, torch.bfloat16, "q")
     _require(kv_pool, torch.bfloat16, "kv_pool")
     _require(block_tables, torch.int32, "block_tables")
@@ -309,7 +311,8 @@ def pa_decode_append(out, q, kv_pool, key, value, slot_mapping, block_tables, se
     [B, Hkv, D], slot_mapping [B]) and pa_decode, in one pass."""
     import torch
 
-    for t, dt, n in ((out, torch.bfloat16, "out"), (q, torch.bfloat16, "q"), (kv_pool, torch.bfloat16, "kv_pool"),
+    _require(out, torch.bfloat16, "out", pinned_ok=True)
+    for t, dt, n in ((q, torch.bfloat16, "q"), (kv_pool, torch.bfloat16, "kv_pool"),
                      (key, torch.bfloat16, "key"), (value, torch.bfloat16, "value"),
                      (slot_mapping, torch.int64, "slot_mapping"), (block_tables, torch.int32, "block_tables"),
                      (seq_lens, torch.int32, "seq_lens")):

@@ -1466,6 +1466,8 @@ static int decode_impl(pa_bf16* out, const pa_bf16* q, const pa_bf16* kv_pool,
   if (!a16(out) || !a16(q) || !a16(kv_pool) || (reinterpret_cast<uintptr_t>(block_tables) & 3u) ||
       (reinterpret_cast<uintptr_t>(seq_lens) & 3u))
     return fail(PA_ERR_INVALID, "pa_decode: misaligned pointer");
+  rc = check_output_pointer(out, "pa_decode");
+  if (rc != PA_OK) return rc;
   bool fused = new_k != nullptr;
   if (fused) {
     if (!new_v || !new_slots) return fail(PA_ERR_INVALID, "pa_decode_append: NULL new_v or slot_mapping");
@@ -1623,6 +1625,8 @@ static int decode_contiguous_impl(pa_bf16* out, const pa_bf16* q, const pa_bf16*
   auto a16 = [](const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; };
   if (!a16(out) || !a16(q) || !a16(kv_cache) || (reinterpret_cast<uintptr_t>(seq_lens) & 3u))
     return fail(PA_ERR_INVALID, "pa_decode_contiguous: misaligned pointer");
+  rc = check_output_pointer(out, "pa_decode_contiguous");
+  if (rc != PA_OK) return rc;
   const int group = hq / hkv;
   if (variant == PA_DECODE_AUTO) variant = kMma;
   if (variant != kCudaCore && variant != kMma)

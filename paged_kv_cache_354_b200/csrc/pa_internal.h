@@ -19,6 +19,14 @@ inline int ok() { return PA_OK; }
 // once per device).  Returns nullptr and records a message on failure.
 int32_t* device_error_word();
 
+// Where a kernel may store its output: device (or managed) memory, or
+// page-locked host memory that the device addresses at the same pointer
+// (cudaHostAlloc / cudaHostRegister under unified addressing), which the
+// kernels then write across PCIe as each result is final.  Pageable host
+// memory and pointers CUDA does not know are refused with PA_ERR_INVALID
+// (a kernel store there would fault).  `who` names the call in the message.
+int check_output_pointer(const void* out, const char* who);
+
 // Streaming multiprocessor count of the current device (cached).
 int sm_count();
 

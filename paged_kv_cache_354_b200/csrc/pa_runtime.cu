@@ -34,6 +34,25 @@ int fail(int status, const char* fmt, ...) {
   return status;
 }
 
+int check_output_pointer(const void* out, const char* who) {
+  cudaPointerAttributes at;
+  const cudaError_t e = cudaPointerGetAttributes(&at, out);
+  if (e != cudaSuccess) {
+    cudaGetLastError();
+    return fail(PA_ERR_INVALID, "%s: out is not a CUDA-visible pointer (%s)", who, cudaGetErrorString(e));
+  }
+  switch (at.type) {
+    case cudaMemoryTypeDevice:
+    case cudaMemoryTypeManaged:
+      return PA_OK;
+    case cudaMemoryTypeHost:
+      if (at.devicePointer == out) return PA_OK;
+      return fail(PA_ERR_INVALID, "%s: out is pinned host memory mapped at another device address", who);
+    default:
+      return fail(PA_ERR_INVALID, "%s: out is pageable host memory; pass device or pinned host memory", who);
+  }
+}
+
 static int current_device(int* dev) {
   cudaError_t e = cudaGetDevice(dev);
   if (e != cudaSuccess) {

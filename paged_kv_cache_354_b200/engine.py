@@ -151,34 +151,52 @@ class PagedDecodeCache:
             pa_copy_blocks(self.pool, self.s_pairs[:npairs])
         self.graph.replay()
 
-    def capture_steps(self, out, h_out):
+    def capture_steps(self, out, h_out, zero_copy=True):
         """Record, for every staging buffer j, a whole step as one CUDA graph:
-        the upload of buffer j, the fused cache write + decode + merge, and the
-        copy of ``out`` into the pinned host tensor ``h_out``.  Needs the graph
-        of ``capture`` (used for steps with copy-on-write pairs, whose copies
-        must run between the upload and the decode)."""
+        the upload of buffer j and the fused cache write + decode + merge,
+        with the output landing in the pinned host tensor ``h_out``.
+
+        zero_copy: the kernels store the output straight into ``h_out``
+        across PCIe as each (request, head) row becomes final, so the rows
+        stream to the host while the decode still runs and only the merged
+        rows are left at its end.  Otherwise the kernels write ``out`` on the
+        device and the graph ends with one device-to-host copy of it.  Both
+        sets of graphs may be recorded; ``replay_step`` uses the one named,
+        or the last recorded.  Needs the graph of ``capture`` (its eager
+        warm-up); steps with copy-on-write pairs run eagerly, since the
+        copies must come between the upload and the decode."""
         assert self.graph is not None, "capture() first"
-        self._out, self._h_out = out, h_out
-        self.step_graphs = []
+        self._out, self._h_out, self._zero_copy = out, h_out, zero_copy
+        graphs = []
         for j in range(len(self.h_stage)):
             g = torch.cuda.CUDAGraph()
             with torch.cuda.graph(g):
                 self.d_stage.copy_(self.h_stage[j], non_blocking=True)
-                self._device_step(out)
-                h_out.copy_(out, non_blocking=True)
-            self.step_graphs.append(g)
+                self._device_step(h_out if zero_copy else out)
+                if not zero_copy:
+                    h_out.copy_(out, non_blocking=True)
+            graphs.append(g)
+        if not hasattr(self, "step_graphs"):
+            self.step_graphs = {}
+        self.step_graphs[bool(zero_copy)] = graphs
+        return graphs
 
-    def replay_step(self, j, npairs):
+    def replay_step(self, j, npairs, zero_copy=None):
         """A whole staged step (asynchronous): one graph launch, or, with
-        copy-on-write pairs, the upload, the copies, the decode graph and the
-        output copy in turn.  ``h_out`` holds the output once the stream is
+        copy-on-write pairs, the upload, the copies and the decode launched
+        one by one.  ``h_out`` holds the output once the stream is
         synchronised."""
+        zc = self._zero_copy if zero_copy is None else bool(zero_copy)
         if npairs:
             self.upload(j)
-            self.replay(npairs)
-            self._h_out.copy_(self._out, non_blocking=True)
+            pa_copy_blocks(self.pool, self.s_pairs[:npairs])
+            if zc:
+                self._device_step(self._h_out)
+            else:
+                self._device_step(self._out)
+                self._h_out.copy_(self._out, non_blocking=True)
         else:
-            self.step_graphs[j].replay()
+            self.step_graphs[zc][j].replay()
 
     # -------------------------------------------------------------- device
     def run(self, q, k_new, v_new, out, slots, tables, lens, pairs=None, max_seq_len=None):

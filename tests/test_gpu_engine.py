@@ -95,11 +95,14 @@ def test_graph_replayed_steps_match_oracle(schedule):
     assert pk.pa_device_error() == 0
 
 
-def test_whole_step_graphs_match_oracle():
-    """capture_steps: upload, fused decode and output copy as one graph per
-    staging buffer (steps with copy-on-write pairs -- here step 3 -- take the
-    eager upload and copies); every step's host output equals the oracle's
-    replay, and the pool equals the oracle's bit for bit."""
+@pytest.mark.parametrize("zero_copy", [True, False])
+def test_whole_step_graphs_match_oracle(zero_copy):
+    """capture_steps: upload and fused decode as one graph per staging
+    buffer, the output reaching pinned host memory straight from the kernels
+    (zero_copy) or through a device-to-host copy in the graph (steps with
+    copy-on-write pairs -- here step 3 -- run eagerly); every step's host
+    output equals the oracle's replay, and the pool equals the oracle's bit
+    for bit."""
     dev = torch.device("cuda", torch.cuda.current_device())
     hq, hkv, d, bs, sets = 8, 2, 128, 16, 3
     nb = 200
@@ -135,7 +138,7 @@ def test_whole_step_graphs_match_oracle():
     cache.upload(0)
     pk.pa_copy_blocks(cache.pool, cache.s_pairs[:npairs])
     cache.capture(out)  # its warm-up performs step 0
-    cache.capture_steps(out, h_out)
+    cache.capture_steps(out, h_out, zero_copy=zero_copy)
     torch.cuda.synchronize()
     seen = 0
     for step in range(7):
