@@ -40,6 +40,8 @@ namespace pa {
 constexpr int kConsumerWarps = 4;
 constexpr int kThreads = (kConsumerWarps + 1) * 32;
 constexpr int kMaxGroup = 8;
+// The widest column count the default variant gives to the tcgen05 consumer.
+constexpr int kTcAutoMaxCols = 16;
 constexpr float kRescaleSlack = 8.f;  // log2 units: probabilities stay <= 256
 constexpr unsigned kFull = 0xffffffffu;
 
@@ -1484,16 +1486,17 @@ static int decode_impl(pa_bf16* out, const pa_bf16* q, const pa_bf16* kv_pool,
     return fail(PA_ERR_UNSUPPORTED, "multi-token decode has the tensor-core variants only");
   // tensor cores for every group: at scale mma.sync beats the CUDA-core
   // consumer even where the group leaves most of the 8-wide tile empty
-  // (g = 1, 2); from 9 to 16 columns the tcgen05 consumer takes over
+  // (g = 1, 2); from 9 to kTcAutoMaxCols columns the tcgen05 consumer takes over
   if (variant == PA_DECODE_AUTO)
-    variant = (group * qtok > kMaxGroup && tc_decode_supported(d, bs, group * qtok)) ? kTc : kMma;
+    variant = (group * qtok > kMaxGroup && group * qtok <= kTcAutoMaxCols &&
+               tc_decode_supported(d, bs, group * qtok)) ? kTc : kMma;
   if (variant == kCudaCore && group != 1 && group != 2 && group != 4)
     return fail(PA_ERR_UNSUPPORTED, "pa_decode: CUDA-core variant has no group size %d", group);
   if (variant != kCudaCore && variant != kMma && variant != kTc)
     return fail(PA_ERR_INVALID, "pa_decode: unknown variant %d", variant);
   if (variant == kTc) {  // the tcgen05 consumer exists on the balanced schedule only
     if (!tc_decode_supported(d, bs, group * qtok))
-      return fail(PA_ERR_UNSUPPORTED, "pa_decode: the tcgen05 variant takes 1..16 columns, not %d", group * qtok);
+      return fail(PA_ERR_UNSUPPORTED, "pa_decode: the tcgen05 variant takes 1..32 columns, not %d", group * qtok);
     if (partition_tokens > 0)
       return fail(PA_ERR_UNSUPPORTED, "pa_decode: the tcgen05 variant runs on the balanced schedule only");
     partition_tokens = kForceBalanced;

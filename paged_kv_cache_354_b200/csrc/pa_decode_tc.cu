@@ -1,6 +1,9 @@
 // Balanced paged decode with a tcgen05 (tensor memory) consumer, for wide
 // column counts: GQA groups of 9..32 query heads per KV head, or several
 // query tokens per request (columns = query tokens x group, up to 32).
+// Columns come in halves of 16: every MMA has N = 16, every tensor-memory
+// access is 16 columns wide and every P tile 32 bytes wide; 17..32 columns
+// run two halves on each loaded tile.
 //
 // What it computes is pa_decode's (quiz page "PagedAttention (vLLM)", code
 // sketch "Conceptual: PagedAttention block lookup": keys and values of
@@ -16,15 +19,17 @@
 //    block as [8-row group][64-dim slab][row][64 dims] (128-byte swizzle), so
 //    in the tile the 8-token groups of every slab sit at one uniform stride
 //    and the tile is a canonical tensor-core operand;
-//  * one thread issues S^T = K Q^T (M = 128 tokens, N = 16 or 32 columns,
-//    K = head dim) into tensor memory, then O^T += V^T P^T (M = head dim,
-//    N = columns, K = the tile's tokens) into a tensor-memory accumulator
-//    that stays there for the whole (request, head) segment;
-//  * four softmax warps each own 32 token rows of S^T (one row per thread,
-//    all columns in registers): mask, online max with a lagging kept max,
-//    probabilities rounded to bf16 into shared memory (the MN-major B operand
-//    of the next MMA); at the end of a segment the same warps read O^T (one
-//    head-dim row per thread) and write the output or the fp32 partial.
+//  * one thread issues S^T = K Q^T (M = 128 tokens, N = 16 columns of a
+//    half, K = head dim) into tensor memory, then O^T += V^T P^T (M = head
+//    dim, N = the half's columns, K = the tile's tokens) into a
+//    tensor-memory accumulator per half that stays there for the whole
+//    (request, head) segment;
+//  * four softmax warps per half each own 32 token rows of S^T (one row per
+//    thread, the half's 16 columns in registers): mask, online max with a
+//    lagging kept max, probabilities rounded to bf16 into shared memory (the
+//    MN-major B operand of the next MMA); at the end of a segment the same
+//    warps read the half's O^T (one head-dim row per thread) and write the
+//    output or the fp32 partial.
 //
 // The running max of a column may lag the true one by up to 2^8 (exp2
 // domain), as in the mma.sync kernel: only when some logit of the tile
@@ -50,20 +55,25 @@ namespace {
 #ifndef PA_TC_TILE_TOKENS
 #define PA_TC_TILE_TOKENS 128
 #endif
-constexpr int kTcThreads = 192;      // warp 0 producer, warp 1 MMA, warps 2..5 softmax
-constexpr int kTcSoftmax = 128;      // softmax / epilogue threads
+// warp 0 producer, warp 1 MMA, then four softmax / epilogue warps per
+// 16-column half (one per TMEM lane quadrant)
+constexpr int kTcSoftmax = 128;      // softmax / epilogue threads of one half
+template <int NH>
+__host__ __device__ constexpr int tc_threads() { return 64 + kTcSoftmax * NH; }
 constexpr int kTcTileTokens = PA_TC_TILE_TOKENS;
 constexpr int kTcRows = 128;         // M of S^T = K Q^T
 constexpr int kTcRingBytes = 196608; // K and V tiles in flight
 static_assert(kTcTileTokens % 32 == 0 && kTcTileTokens <= kTcRows, "tile of 32, 64, 96 or 128 tokens");
 constexpr float kTcSlack = 8.f;      // log2 units: probabilities stay <= 256
-constexpr int kTcMaxCols = 16;       // (token, head) columns per KV head
+constexpr int kTcHalf = 16;          // columns per MMA (N), per TMEM access, per P tile
+constexpr int kTcMaxCols = 32;       // (token, head) columns per KV head: two halves
 
-template <int D, int BS, int N>
+template <int D, int BS, int NH>
 struct TcGeo {
   static_assert(D == 64 || D == 128, "head_dim 64 or 128");
   static_assert(BS == 16 || BS == 32, "block_size 16 or 32");
-  static_assert(N == 16 || N == 32, "16 or 32 columns");
+  static_assert(NH == 1 || NH == 2, "one or two 16-column halves");
+  static constexpr int kCols = kTcHalf * NH;                 // columns the CTA holds per KV head
   static constexpr int kSlabs = D / 64;
   static constexpr int kTileBlocks = kTcTileTokens / BS;
   static constexpr int kChunk = (32 / kTileBlocks) * kTileBlocks;  // table entries per warp load
@@ -71,10 +81,11 @@ struct TcGeo {
   static constexpr int kTileBytes = kTcTileTokens * D * 2;
   static constexpr int kStages = kTcRingBytes / (2 * kTileBytes);  // 3 (D128) or 6 (D64)
   static constexpr int kGroupStride = kSlabs * 1024;         // between 8-token groups of a tile
-  static constexpr int kQSlab = N * 128;                     // one 64-dim slab of Q (N rows)
+  static constexpr int kQSlab = kCols * 128;                 // one 64-dim slab of Q (kCols rows)
   static constexpr int kQBytes = kSlabs * kQSlab;
-  static constexpr int kPRow = N * 2;                        // one token's probabilities
-  static constexpr int kPBytes = kTcRows * kPRow;
+  static constexpr int kPRow = kTcHalf * 2;                  // one token's probabilities in a half
+  static constexpr int kPHalf = kTcRows * kPRow;             // the P tile of one half
+  static constexpr int kPBytes = NH * kPHalf;
   static constexpr int kK = 0;
   static constexpr int kV = kStages * kTileBytes;
   static constexpr int kQ = 2 * kStages * kTileBytes;
@@ -88,15 +99,17 @@ struct TcGeo {
   static constexpr int kNumBars = 4 * kStages + 11 + kInfoSlots;
   static constexpr int kInfo = (kBar + 8 * kNumBars + 15) & ~15;  // TileInfo[kInfoSlots]
   static constexpr int kMisc = kInfo + 32 * kInfoSlots;  // tmem base, abort, last_k[S], last_v[S], last_q[2]
-  static constexpr int kRedMax = (kMisc + 8 + 8 * kStages + 8 + 15) & ~15;  // float [4][N]
-  static constexpr int kRedSum = kRedMax + 4 * N * 4;                     // float [4][N]
-  static constexpr int kTotal = kRedSum + 4 * N * 4;
+  static constexpr int kRedMax = (kMisc + 8 + 8 * kStages + 8 + 15) & ~15;  // float [4][kCols]
+  static constexpr int kRedSum = kRedMax + 4 * kCols * 4;                 // float [4][kCols]
+  static constexpr int kTotal = kRedSum + 4 * kCols * 4;
   static constexpr int kDynamic = kTotal + 1024;  // 1024-byte alignment slack
   static_assert(kDynamic <= 232448, "shared memory per CTA");
   static_assert(kQSlab % 1024 == 0 && kPBytes % 1024 == 0 && kTileBytes % 1024 == 0, "swizzle atoms");
   // the last K tile's M = 128 rows may run (kTcRows - kTcTileTokens) rows into the V ring
   static_assert(kV - kTileBytes + kTcRows * D * 2 <= kTotal, "S^T rows past the tile stay in shared memory");
-  static constexpr uint32_t kTmemCols = 128;  // S^T double buffer (2N) + O^T (N)
+  // S^T double buffer (2 kCols) + O^T (kCols): columns [0, 3 kCols)
+  static constexpr uint32_t kTmemCols = 128;
+  static_assert(3 * kCols <= static_cast<int>(kTmemCols), "tensor memory columns");
 };
 
 // Published by the producer for every tile it loads, read by the MMA and
@@ -115,61 +128,54 @@ constexpr int kLast = 2;      // last tile of a segment
 constexpr int kComplete = 4;  // the segment covers its whole (request, head)
 constexpr int kFinal = 8;     // last tile of the CTA
 
-__device__ __forceinline__ bool softmax_any(bool pred) {
+// Named barrier `id` (1 + half) over the 128 softmax threads of one half.
+__device__ __forceinline__ bool softmax_any(bool pred, uint32_t id) {
   __syncwarp();  // an aligned barrier: the warp arrives converged
   uint32_t r;
   asm volatile(
       "{\n\t.reg .pred p, q;\n\t"
       "setp.ne.u32 p, %1, 0;\n\t"
-      "bar.red.or.pred q, 1, 128, p;\n\t"
+      "bar.red.or.pred q, %2, 128, p;\n\t"
       "selp.u32 %0, 1, 0, q;\n\t}"
       : "=r"(r)
-      : "r"(pred ? 1u : 0u)
+      : "r"(pred ? 1u : 0u), "r"(id)
       : "memory");
   return r != 0;
 }
 
-__device__ __forceinline__ void softmax_sync() {
+__device__ __forceinline__ void softmax_sync(uint32_t id) {
   __syncwarp();
-  asm volatile("bar.sync 1, 128;" ::: "memory");
+  asm volatile("bar.sync %0, 128;" ::"r"(id) : "memory");
 }
 
-// Warp-wide TMEM accesses.  They are .sync.aligned: the warp reconverges
-// first (the bounded mbarrier waits before them let lanes leave their spin
-// loops at different iterations), and a load returns only after its wait.
-template <int N>
-__device__ __forceinline__ void tmem_load(uint32_t taddr, uint32_t (&r)[N]) {
+// Warp-wide TMEM accesses of 16 columns.  They are .sync.aligned: the warp
+// reconverges first (the bounded mbarrier waits before them let lanes leave
+// their spin loops at different iterations), and a load returns only after
+// its wait.
+__device__ __forceinline__ void tmem_load16(uint32_t taddr, uint32_t (&r)[kTcHalf]) {
   __syncwarp();
-  if constexpr (N == 32) {
-    tc::tmem_ld_x32(taddr, r);
-    tc::wait_ld_x32(r);
-  } else {
-    tc::tmem_ld_x16(taddr, r);
-    tc::wait_ld_x16(r);
-  }
+  tc::tmem_ld_x16(taddr, r);
+  tc::wait_ld_x16(r);
 }
-template <int N>
-__device__ __forceinline__ void tmem_store(uint32_t taddr, const uint32_t (&r)[N]) {
+__device__ __forceinline__ void tmem_store16(uint32_t taddr, const uint32_t (&r)[kTcHalf]) {
   __syncwarp();
-  if constexpr (N == 32) tc::tmem_st_x32(taddr, r);
-  else tc::tmem_st_x16(taddr, r);
+  tc::tmem_st_x16(taddr, r);
   tc::wait_st();
 }
 
-// Column-wise reduction across the warp's 32 lanes of v[0..N): afterwards
-// lane c holds the result for column c mod N.  Each step halves the columns
-// a lane keeps and hands the other half to its partner.
-template <int N, bool kMax>
-__device__ __forceinline__ float warp_columns(float (&v)[N], int lane) {
-  if constexpr (N == 16) {
+// Column-wise reduction of 16 columns v[0..16) across the warp's 32 lanes:
+// afterwards lane c holds the result for column c mod 16.  The lanes l and
+// l + 16 first combine every column, then each step halves the columns a
+// lane keeps and hands the other half to its partner.
+template <bool kMax>
+__device__ __forceinline__ float warp_columns(float (&v)[kTcHalf], int lane) {
 #pragma unroll
-    for (int c = 0; c < 16; ++c) {
-      const float o = __shfl_xor_sync(kFullMask, v[c], 16);
-      v[c] = kMax ? fmaxf(v[c], o) : v[c] + o;
-    }
+  for (int c = 0; c < kTcHalf; ++c) {
+    const float o = __shfl_xor_sync(kFullMask, v[c], 16);
+    v[c] = kMax ? fmaxf(v[c], o) : v[c] + o;
   }
 #pragma unroll
-  for (int off = N / 2; off >= 1; off >>= 1) {
+  for (int off = kTcHalf / 2; off >= 1; off >>= 1) {
     const bool upper = (lane & off) != 0;
 #pragma unroll
     for (int c = 0; c < off; ++c) {
@@ -182,12 +188,15 @@ __device__ __forceinline__ float warp_columns(float (&v)[N], int lane) {
   return v[0];
 }
 
-template <int D, int BS, int N>
-__global__ void __launch_bounds__(kTcThreads, 1)
+template <int D, int BS, int NH>
+__global__ void __launch_bounds__(tc_threads<NH>(), 1)
     paged_decode_tc_kernel(const __grid_constant__ CUtensorMap kv_map, const __grid_constant__ CUtensorMap q_map,
                            const DecodeArgs a, int batch) {
-  using G = TcGeo<D, BS, N>;
+  using G = TcGeo<D, BS, NH>;
   constexpr int S = G::kStages;
+  constexpr int NC = G::kCols;  // columns held: 16 per half
+  constexpr int H16 = kTcHalf;
+  constexpr int kThreads = tc_threads<NH>();
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw_base = smem_u32(smem_raw);
   const uint32_t pad = ((raw_base + 1023u) & ~1023u) - raw_base;
@@ -240,7 +249,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       mbar_init(q_full(j), 1);
       mbar_init(q_empty(j), 1);
       mbar_init(s_full(j), 1);
-      mbar_init(p_full(j), kTcSoftmax);
+      mbar_init(p_full(j), kTcSoftmax * NH);
       last_q[j] = -1;
     }
     mbar_init(pv_done(0), 1);
@@ -261,9 +270,9 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   // per-request block-count prefix sums, in the still idle K ring
   int* prefix = reinterpret_cast<int*>(smem + G::kK);
   int* scan = prefix + ((batch + 1 + 3) & ~3);
-  block_count_prefix<BS, kTcThreads>(prefix, scan, batch, a, blockIdx.x == 0);
+  block_count_prefix<BS, kThreads>(prefix, scan, batch, a, blockIdx.x == 0);
   if (blockIdx.x == 0)
-    for (int i = threadIdx.x; i <= batch; i += kTcThreads) a.stream_prefix[i] = prefix[i];
+    for (int i = threadIdx.x; i <= batch; i += kThreads) a.stream_prefix[i] = prefix[i];
   const long long total = static_cast<long long>(hkv) * prefix[batch];
   const long long u_begin = stream_begin(total, blockIdx.x, ctas);
   const long long u_end = stream_begin(total, blockIdx.x + 1, ctas);
@@ -411,24 +420,30 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     } else if (warp == 1) {
       // --------------------------------------------------------- MMA issue
       if (lane == 0) {
-        constexpr uint32_t kIdS = tc::idesc_bf16(128, N, false, false);
-        constexpr uint32_t kIdO = tc::idesc_bf16(128, N, true, true);
-        constexpr uint64_t kPSwizzle = N == 32 ? tc::kSwizzle64B : tc::kSwizzle32B;
-        // S^T (tile i) = K Q^T over the head dim, 16 dims per instruction
+        constexpr uint32_t kIdS = tc::idesc_bf16(128, H16, false, false);
+        constexpr uint32_t kIdO = tc::idesc_bf16(128, H16, true, true);
+        // S^T (tile i) = K Q^T over the head dim, 16 dims per instruction;
+        // half h2 multiplies Q rows [16 h2, 16 h2 + 16) (two 8-row groups
+        // further on) into its own 16 TMEM columns
         auto issue_s = [&](int i, const TileInfo& t) {
           const uint32_t kt = sbase + G::kK + (i % S) * G::kTileBytes;
           const uint32_t qt = sbase + G::kQ + (t.qseg & 1) * G::kQBytes;
-          const uint32_t d = tmem + (i & 1) * N;
+          const uint32_t d = tmem + (i & 1) * NC;
 #pragma unroll
           for (int ks = 0; ks < D / 16; ++ks) {
             const int x = ks >> 2, kk = ks & 3;
             const uint64_t ad = tc::smem_desc(kt + x * 1024 + kk * 32, 16, G::kGroupStride, tc::kSwizzle128B);
-            const uint64_t bd = tc::smem_desc(qt + x * G::kQSlab + kk * 32, 16, 1024, tc::kSwizzle128B);
-            tc::mma_bf16(d, ad, bd, kIdS, ks > 0 ? 1u : 0u);
+#pragma unroll
+            for (int h2 = 0; h2 < NH; ++h2) {
+              const uint64_t bd =
+                  tc::smem_desc(qt + x * G::kQSlab + h2 * 2048 + kk * 32, 16, 1024, tc::kSwizzle128B);
+              tc::mma_bf16(d + h2 * H16, ad, bd, kIdS, ks > 0 ? 1u : 0u);
+            }
           }
         };
-        // O^T += V^T P^T over the tile's real tokens, 16 per instruction;
-        // head dim 64 makes rows 64..127 repeat rows 0..63 (unused)
+        // O^T += V^T P^T over the tile's real tokens, 16 per instruction, one
+        // accumulator per half; head dim 64 makes rows 64..127 repeat rows
+        // 0..63 (unused)
         auto issue_pv = [&](int i, const TileInfo& t) {
           const uint32_t vt = sbase + G::kV + (i % S) * G::kTileBytes;
           const uint32_t pt = sbase + G::kP + (i & 1) * G::kPBytes;
@@ -436,8 +451,12 @@ __global__ void __launch_bounds__(kTcThreads, 1)
           for (int kk = 0; kk < steps; ++kk) {
             const uint64_t ad =
                 tc::smem_desc(vt + 2 * kk * G::kGroupStride, D == 128 ? 1024 : 0, G::kGroupStride, tc::kSwizzle128B);
-            const uint64_t bd = tc::smem_desc(pt + kk * 16 * G::kPRow, 8192, 8 * G::kPRow, kPSwizzle);
-            tc::mma_bf16(tmem + 2 * N, ad, bd, kIdO, ((t.flags & kFirst) && kk == 0) ? 0u : 1u);
+#pragma unroll
+            for (int h2 = 0; h2 < NH; ++h2) {
+              const uint64_t bd =
+                  tc::smem_desc(pt + h2 * G::kPHalf + kk * 16 * G::kPRow, 8192, 8 * G::kPRow, tc::kSwizzle32B);
+              tc::mma_bf16(tmem + 2 * NC + h2 * H16, ad, bd, kIdO, ((t.flags & kFirst) && kk == 0) ? 0u : 1u);
+            }
           }
         };
         auto give_up = [&]() {
@@ -519,19 +538,24 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       __syncwarp();
     } else {
       // ---------------------------------------------- softmax and epilogue
+      // four warps per half: half h2 owns columns [16 h2, 16 h2 + 16), its
+      // S^T and O^T columns in TMEM and its P tile
+      const int h2 = (warp - 2) >> 2;
+      const uint32_t bar_id = 1 + h2;   // the half's named barrier
+      const int c0 = h2 * H16;          // its first column
       const int qd = warp & 3;          // TMEM lane quadrant of this warp
       const int row = 32 * qd + lane;   // token row of S^T, head-dim row of O^T
       float* red_max = reinterpret_cast<float*>(smem + G::kRedMax);
       float* red_sum = reinterpret_cast<float*>(smem + G::kRedSum);
       const size_t q_tok_heads = static_cast<size_t>(a.num_q_heads);
-      float m[N], l[N];
+      float m[H16], l[H16];  // this half's columns
       int i = 0;
       bool bad = false;  // a wait of this thread ran out; checked uniformly at the next tile
       while (true) {
         const int s = i % S;
         if (!bad) bad = !mbar_wait(info_full(i % G::kInfoSlots), (i / G::kInfoSlots) & 1);
         if (!bad) bad = !mbar_wait(s_full(i & 1), (i >> 1) & 1);
-        if (softmax_any(bad || *abort_flag != 0)) {  // uniform: all four warps leave together
+        if (softmax_any(bad || *abort_flag != 0, bar_id)) {  // uniform: the half's four warps leave together
           if (bad) {
             flag_error(a.err, PA_DEVERR_WAIT_TIMEOUT);
             *abort_flag = 1;
@@ -540,11 +564,11 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         }
         const TileInfo t = info[i % G::kInfoSlots];
         tc::fence_after_sync();
-        uint32_t sr[N];
-        tmem_load<N>(tc::tmem_addr(tmem, 32 * qd, (i & 1) * N), sr);
+        uint32_t sr[H16];
+        tmem_load16(tc::tmem_addr(tmem, 32 * qd, (i & 1) * NC + c0), sr);
         if (t.flags & kFirst) {
 #pragma unroll
-          for (int c = 0; c < N; ++c) {
+          for (int c = 0; c < H16; ++c) {
             m[c] = -INFINITY;
             l[c] = 0.f;
           }
@@ -552,51 +576,52 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         // column c = (query token c / g, head c % g) sees positions <= len - qtok + c / g
         const int pos = t.pos0 + row;
         const bool real = row < t.nblk * BS;
-        const int cmin = real ? max(0, g * (pos - (t.len - a.qtok))) : N;
-        float sv[N];
+        const int cmin = real ? max(0, g * (pos - (t.len - a.qtok))) : NC;
+        float sv[H16];
         bool over = false;
 #pragma unroll
-        for (int c = 0; c < N; ++c) {
-          const bool vis = c >= cmin && c < cols;
+        for (int c = 0; c < H16; ++c) {
+          const bool vis = c0 + c >= cmin && c0 + c < cols;
           sv[c] = vis ? __uint_as_float(sr[c]) * a.scale_log2 : -INFINITY;
           over |= sv[c] > m[c] + kTcSlack;  // true while m = -inf
         }
-        if (softmax_any(over)) {
+        if (softmax_any(over, bar_id)) {
           // exact column maxima over the tile's 128 rows
-          float mx[N];
+          float mx[H16];
 #pragma unroll
-          for (int c = 0; c < N; ++c) mx[c] = sv[c];
-          const float wmax = warp_columns<N, true>(mx, lane);
-          if (lane < N) red_max[qd * N + lane] = wmax;
-          softmax_sync();
+          for (int c = 0; c < H16; ++c) mx[c] = sv[c];
+          const float wmax = warp_columns<true>(mx, lane);
+          if (lane < H16) red_max[qd * NC + c0 + lane] = wmax;
+          softmax_sync(bar_id);
           bool rescale = false;
-          float alpha[N];
+          float alpha[H16];
 #pragma unroll
-          for (int c = 0; c < N; ++c) {
-            const float mn = fmaxf(fmaxf(m[c], fmaxf(red_max[c], red_max[N + c])),
-                                   fmaxf(red_max[2 * N + c], red_max[3 * N + c]));
+          for (int c = 0; c < H16; ++c) {
+            const float mn = fmaxf(fmaxf(m[c], fmaxf(red_max[c0 + c], red_max[NC + c0 + c])),
+                                   fmaxf(red_max[2 * NC + c0 + c], red_max[3 * NC + c0 + c]));
             alpha[c] = (m[c] == -INFINITY) ? 0.f : exp2f(m[c] - mn);
             rescale |= (m[c] != -INFINITY) && (mn != m[c]);
             l[c] *= alpha[c];
             m[c] = mn;
           }
-          softmax_sync();  // red_max is read; it may be written again
+          softmax_sync(bar_id);  // red_max is read; it may be written again
           if (rescale && !(t.flags & kFirst)) {
             // O^T holds the sum through tile i-1: rescale it in place
             if (!bad) bad = !mbar_wait(pv_done((i - 1) & 1), ((i - 1) >> 1) & 1);
             tc::fence_after_sync();
-            uint32_t o[N];
-            tmem_load<N>(tc::tmem_addr(tmem, 32 * qd, 2 * N), o);
+            uint32_t o[H16];
+            const uint32_t oaddr = tc::tmem_addr(tmem, 32 * qd, 2 * NC + c0);
+            tmem_load16(oaddr, o);
 #pragma unroll
-            for (int c = 0; c < N; ++c) o[c] = __float_as_uint(__uint_as_float(o[c]) * alpha[c]);
-            tmem_store<N>(tc::tmem_addr(tmem, 32 * qd, 2 * N), o);
+            for (int c = 0; c < H16; ++c) o[c] = __float_as_uint(__uint_as_float(o[c]) * alpha[c]);
+            tmem_store16(oaddr, o);
           }
         }
-        // probabilities (bf16) -> P row of this token; the sums take the
-        // rounded values the MMA multiplies
-        const uint32_t prow = sbase + G::kP + (i & 1) * G::kPBytes + row * G::kPRow;
+        // probabilities (bf16) -> this half's P row of this token (32 bytes);
+        // the sums take the rounded values the MMA multiplies
+        const uint32_t prow = sbase + G::kP + (i & 1) * G::kPBytes + h2 * G::kPHalf + row * G::kPRow;
 #pragma unroll
-        for (int ch = 0; ch < N / 8; ++ch) {
+        for (int ch = 0; ch < 2; ++ch) {
           uint32_t w[4];
 #pragma unroll
           for (int e = 0; e < 4; ++e) {
@@ -607,14 +632,15 @@ __global__ void __launch_bounds__(kTcThreads, 1)
             l[c] += bf16lo_to_f32(w[e]);
             l[c + 1] += bf16hi_to_f32(w[e]);
           }
-          const int sw = N == 32 ? (ch ^ ((row >> 1) & 3)) : (ch ^ ((row >> 2) & 1));
+          const int sw = ch ^ ((row >> 2) & 1);  // 32-byte swizzle
           asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};" ::"r"(prow + sw * 16), "r"(w[0]), "r"(w[1]),
                        "r"(w[2]), "r"(w[3])
                        : "memory");
         }
         // rows past the request's end inside its last block may hold NaN:
-        // zero their values so P = 0 there contributes exactly 0
-        if (real && pos >= t.len) {
+        // zero their values so P = 0 there contributes exactly 0 (the first
+        // half's warps; the P.V of every half waits for all of them)
+        if (h2 == 0 && real && pos >= t.len) {
           if (!bad) bad = !mbar_wait(v_full(s), (i / S) & 1);
           const uint32_t vrow = sbase + G::kV + s * G::kTileBytes + (row >> 3) * G::kGroupStride + (row & 7) * 128;
 #pragma unroll
@@ -630,28 +656,28 @@ __global__ void __launch_bounds__(kTcThreads, 1)
 
         if (t.flags & kLast) {
           // ---- segment epilogue: column sums over the 128 rows, then O^T
-          float lv[N];
+          float lv[H16];
 #pragma unroll
-          for (int c = 0; c < N; ++c) lv[c] = l[c];
-          const float wsum = warp_columns<N, false>(lv, lane);
-          if (lane < N) red_sum[qd * N + lane] = wsum;
-          softmax_sync();
-          const int cl = lane & (N - 1);
-          const float lsum = red_sum[cl] + red_sum[N + cl] + red_sum[2 * N + cl] + red_sum[3 * N + cl];
-          softmax_sync();  // red_sum is read
+          for (int c = 0; c < H16; ++c) lv[c] = l[c];
+          const float wsum = warp_columns<false>(lv, lane);
+          if (lane < H16) red_sum[qd * NC + c0 + lane] = wsum;
+          softmax_sync(bar_id);
+          const int cl = c0 + (lane & (H16 - 1));  // lane c: the half's column c mod 16
+          const float lsum = red_sum[cl] + red_sum[NC + cl] + red_sum[2 * NC + cl] + red_sum[3 * NC + cl];
+          softmax_sync(bar_id);  // red_sum is read
           if (!bad) bad = !mbar_wait(pv_done(i & 1), (i >> 1) & 1);
           tc::fence_after_sync();
-          uint32_t o[N];
-          tmem_load<N>(tc::tmem_addr(tmem, 32 * qd, 2 * N), o);
+          uint32_t o[H16];
+          tmem_load16(tc::tmem_addr(tmem, 32 * qd, 2 * NC + c0), o);
           tc::fence_before_sync();  // the next segment's first MMA overwrites O^T
           const size_t qrow0 = static_cast<size_t>(t.b) * a.qtok * q_tok_heads + static_cast<size_t>(t.h) * g;
           if (t.flags & kComplete) {
             const float inv_l = lsum > 0.f ? 1.f / lsum : 0.f;  // a token that sees nothing gets 0
-            int tt = 0, j = 0;
+            int tt = c0 / g, j = c0 - (c0 / g) * g;  // (query token, head) of column c0
 #pragma unroll
-            for (int c = 0; c < N; ++c) {
+            for (int c = 0; c < H16; ++c) {
               const float inv = __shfl_sync(kFullMask, inv_l, c);
-              if (c < cols && row < D)
+              if (c0 + c < cols && row < D)
                 a.out[(qrow0 + tt * q_tok_heads + j) * D + row] = __float2bfloat16_rn(__uint_as_float(o[c]) * inv);
               if (++j == g) {
                 j = 0;
@@ -661,14 +687,14 @@ __global__ void __launch_bounds__(kTcThreads, 1)
           } else {
             const size_t prow_part = (static_cast<size_t>(blockIdx.x) * 2 + (t.seg == 0 ? 0 : 1)) * cols;
 #pragma unroll
-            for (int c = 0; c < N; ++c)
-              if (c < cols && row < D) a.part_o[(prow_part + c) * D + row] = __uint_as_float(o[c]);
-            if (qd == 0 && lane < cols) {
+            for (int c = 0; c < H16; ++c)
+              if (c0 + c < cols && row < D) a.part_o[(prow_part + c0 + c) * D + row] = __uint_as_float(o[c]);
+            if (qd == 0 && lane < H16 && c0 + lane < cols) {
               float mc = m[0];
 #pragma unroll
-              for (int c = 1; c < N; ++c) mc = (lane == c) ? m[c] : mc;
-              a.part_m[prow_part + lane] = mc;
-              a.part_l[prow_part + lane] = lsum;
+              for (int c = 1; c < H16; ++c) mc = (lane == c) ? m[c] : mc;
+              a.part_m[prow_part + c0 + lane] = mc;
+              a.part_l[prow_part + c0 + lane] = lsum;
             }
           }
         }
@@ -701,25 +727,25 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   }
 }
 
-template <int D, int BS, int N>
+template <int D, int BS, int NH>
 int launch_tc(const CUtensorMap& kv_map, const CUtensorMap& q_map, const DecodeArgs& a, int batch, int ctas,
               cudaStream_t st) {
-  using G = TcGeo<D, BS, N>;
-  auto kern = paged_decode_tc_kernel<D, BS, N>;
+  using G = TcGeo<D, BS, NH>;
+  auto kern = paged_decode_tc_kernel<D, BS, NH>;
   int rc = set_smem_attr(reinterpret_cast<const void*>(kern), G::kDynamic);
   if (rc != PA_OK) return rc;
-  PA_CUDA_TRY(launch_pdl(kern, dim3(static_cast<unsigned>(ctas)), dim3(kTcThreads), G::kDynamic, st, kv_map, q_map,
-                         a, batch));
+  PA_CUDA_TRY(launch_pdl(kern, dim3(static_cast<unsigned>(ctas)), dim3(tc_threads<NH>()), G::kDynamic, st, kv_map,
+                         q_map, a, batch));
   return PA_OK;
 }
 
-// Up to 16 (token, head) columns: one 16-column MMA tile.  (A 32-column
-// build raised an illegal-instruction fault at the Llama-3-8B lengths whose
-// cause is not yet found; it is not compiled.)
+// Up to 16 (token, head) columns: one half; 17..32: two halves sharing
+// every loaded tile.
 template <int D, int BS>
 int launch_tc_cols(const CUtensorMap& kv_map, const CUtensorMap& q_map, const DecodeArgs& a, int batch, int ctas,
                    cudaStream_t st) {
-  return launch_tc<D, BS, 16>(kv_map, q_map, a, batch, ctas, st);
+  if (a.cols <= kTcHalf) return launch_tc<D, BS, 1>(kv_map, q_map, a, batch, ctas, st);
+  return launch_tc<D, BS, 2>(kv_map, q_map, a, batch, ctas, st);
 }
 
 }  // namespace

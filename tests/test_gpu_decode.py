@@ -78,11 +78,12 @@ def test_split_k_partitions(partition_blocks, variant):
     [40000],                   # one request cut across every CTA
     [17, 40000, 0, 5, 2048],   # mixed, with a request split many ways
 ])
-@pytest.mark.parametrize("variant", ["mma", "cuda_core", "tcgen05"])
+@pytest.mark.parametrize("variant", ["mma", "cuda_core", "tcgen05", "tcgen05_two_halves"])
 def test_balanced_schedule_edges(lens, variant):
-    hq, hkv = {"mma": (8, 2), "cuda_core": (4, 4), "tcgen05": (32, 2)}[variant]
-    for d in (64, 128) if variant == "tcgen05" else (64,):
-        check(lens, hq, hkv, d, 16, seed=60 + len(lens), variant=variant, partition_tokens=pk.PA_SCHEDULE_BALANCED)
+    hq, hkv = {"mma": (8, 2), "cuda_core": (4, 4), "tcgen05": (32, 2), "tcgen05_two_halves": (58, 2)}[variant]
+    v = "tcgen05" if variant.startswith("tcgen05") else variant
+    for d in (64, 128) if v == "tcgen05" else (64,):
+        check(lens, hq, hkv, d, 16, seed=60 + len(lens), variant=v, partition_tokens=pk.PA_SCHEDULE_BALANCED)
 
 
 def test_balanced_matches_partition_grid():
@@ -106,21 +107,23 @@ def test_wide_groups(d, bs, schedule, hq, hkv, variant):
 
 
 @pytest.mark.parametrize("d,bs", [(128, 16), (128, 32), (64, 16), (64, 32)])
-@pytest.mark.parametrize("hq,hkv", [(2, 2), (8, 2), (18, 2), (26, 2), (32, 2), (16, 1), (96, 8)])
+@pytest.mark.parametrize("hq,hkv", [(2, 2), (8, 2), (18, 2), (26, 2), (32, 2), (16, 1), (96, 8),
+                                    (34, 2), (48, 2), (62, 2), (64, 2), (32, 1), (256, 8)])
 def test_tcgen05_variant(d, bs, hq, hkv):
-    """The tcgen05 consumer for 1..16 (token, head) columns (one 16-column
-    MMA tile): 128-token tiles with ragged ends, tiles cut between CTAs,
-    requests of exactly one tile, NaN in every unused pool row."""
+    """The tcgen05 consumer for 1..32 (token, head) columns (one 16-column
+    half, or two sharing each tile from 17 columns): 128-token tiles with
+    ragged ends, tiles cut between CTAs, requests of exactly one tile, NaN
+    in every unused pool row."""
     check(RAGGED + [2000, 129, 128, 127, 4111], hq, hkv, d, bs, seed=300 + d + bs + hq + hkv, variant="tcgen05")
 
 
-def test_tcgen05_rejects_more_than_16_columns():
-    q, pool, _, (t, l) = make_case([40, 70], 34, 2, 128, 16, seed=301)
+def test_tcgen05_rejects_more_than_32_columns():
+    q, pool, _, (t, l) = make_case([40, 70], 68, 2, 128, 16, seed=301)
     with pytest.raises(pk.PaError):
         run_decode(q.cuda(), pool.cuda(), t, l, 0.1, pk.PA_DECODE_TCGEN05)
 
 
-@pytest.mark.parametrize("hq,hkv", [(24, 2), (32, 2)])
+@pytest.mark.parametrize("hq,hkv", [(24, 2), (32, 2), (48, 2), (64, 2)])
 def test_tcgen05_matches_mma_sync(hq, hkv):
     """Both tensor-core consumers on the same wide-group inputs: equal up to
     the rounding of their different summation orders."""
@@ -184,14 +187,33 @@ def test_zero_length_request():
     compare(bf16_to_f64(out), want)
 
 
-def test_large_logits():
-    """A large scale makes the softmax nearly one-hot; the online max must hold
-    (for the wide groups: the column maxima and the rescale of O in tensor
-    memory)."""
-    check([77, 500], 8, 2, 128, 16, seed=13, scale=4.0)
-    check([77, 500], 4, 4, 64, 16, seed=14, scale=4.0)
-    check([77, 500, 3000], 32, 2, 128, 16, seed=15, scale=4.0, variant="tcgen05")
-    check([77, 500, 3000], 24, 2, 64, 32, seed=16, scale=4.0, variant="tcgen05")
+@pytest.mark.parametrize("lens,hq,hkv,d,bs,seed,variant", [
+    ([77, 500], 8, 2, 128, 16, 13, "auto"),
+    ([77, 500], 4, 4, 64, 16, 14, "auto"),
+    ([77, 500, 3000], 32, 2, 128, 16, 15, "tcgen05"),
+    ([77, 500, 3000], 24, 2, 64, 32, 16, "tcgen05"),
+    ([77, 500, 3000], 64, 2, 128, 16, 17, "tcgen05"),
+    ([77, 500, 3000], 40, 2, 64, 16, 18, "tcgen05"),
+    ([77, 500, 3000], 64, 2, 128, 16, 17, "mma"),
+])
+def test_large_logits(lens, hq, hkv, d, bs, seed, variant):
+    """Scale 4 (45x the usual 1/sqrt(128)) makes the softmax nearly one-hot;
+    the online max must hold (for the wide groups: the column maxima and the
+    rescale of O in tensor memory).  An output is then nearly one value
+    row, up to ~4.5 in magnitude, and its bf16 rounding alone can reach half
+    a unit in the last place, 2^-8 |out| (0.0176 at 4.5): so here the bound
+    per element is 1e-2 + 2^-8 |want| (the fixed 1e-2 plus that rounding),
+    and the mean stays <= 1e-3."""
+    q, pool, (t_ref, l_ref), (t_cpp, l_cpp) = make_case(lens, hq, hkv, d, bs, seed)
+    want = opa.decode(bf16_to_f64(q), bf16_to_f64(pool), t_ref, l_ref, 4.0)
+    out = run_decode(q.cuda(), pool.cuda(), t_cpp, l_cpp, 4.0, VARIANTS[variant],
+                     pk.PA_SCHEDULE_BALANCED if hq // hkv > 8 else 0)
+    assert pk.pa_device_error() == 0
+    got = bf16_to_f64(out)
+    err = np.abs(got - want)
+    assert np.isfinite(got).all()
+    assert (err <= 1e-2 + 2.0 ** -8 * np.abs(want)).all(), float((err - 2.0 ** -8 * np.abs(want)).max())
+    assert err.mean() <= 1e-3
 
 
 def test_tiny_workload():
@@ -223,19 +245,21 @@ def test_device_checks_flag_bad_inputs():
     assert pk.pa_device_error() == 0  # cleared by the previous read
 
 
-BAD_ID_CASES = [(v, 128, 16, pk.PA_SCHEDULE_BALANCED) for v in ("mma", "cuda_core", "tcgen05")] + \
-    [(v, 128, 16, 64) for v in ("mma", "cuda_core")] + \
-    [(v, 64, 16, pk.PA_SCHEDULE_BALANCED) for v in ("mma", "cuda_core", "tcgen05")] + \
-    [(v, 64, 32, 0) for v in ("mma", "cuda_core", "tcgen05")]
+BAD_ID_CASES = [(v, 128, 16, pk.PA_SCHEDULE_BALANCED, 8) for v in ("mma", "cuda_core", "tcgen05")] + \
+    [(v, 128, 16, 64, 8) for v in ("mma", "cuda_core")] + \
+    [(v, 64, 16, pk.PA_SCHEDULE_BALANCED, 8) for v in ("mma", "cuda_core", "tcgen05")] + \
+    [(v, 64, 32, 0, 8) for v in ("mma", "cuda_core", "tcgen05")] + \
+    [(v, d, 16, pk.PA_SCHEDULE_BALANCED, 40) for v in ("mma", "tcgen05") for d in (64, 128)]
 
 
-@pytest.mark.parametrize("variant,d,bs,schedule", BAD_ID_CASES)
-def test_bad_block_ids_read_zeros(variant, d, bs, schedule):
+@pytest.mark.parametrize("variant,d,bs,schedule,hq", BAD_ID_CASES)
+def test_bad_block_ids_read_zeros(variant, d, bs, schedule, hq):
     """A table entry outside [0, num_blocks) -- past the end or negative --
     reads a block of zeros and flags PA_DEVERR_BLOCK_ID: the output equals the
-    oracle's over a pool whose extra block is all zeros."""
+    oracle's over a pool whose extra block is all zeros.  (Group 20: the
+    paired-warp mma.sync kernel and the tcgen05 consumer's two halves.)"""
     lens = [40, 100, 70]
-    q, pool, (t_ref, l_ref), (t, l) = make_case(lens, 8, 2, d, bs, seed=17 + d + bs)
+    q, pool, (t_ref, l_ref), (t, l) = make_case(lens, hq, 2, d, bs, seed=17 + d + bs)
     nb = pool.shape[0]
     bad = t.copy()
     bad[0, 1] = nb + 5
