@@ -170,7 +170,7 @@ int pa_copy_blocks(pa_bf16* kv_pool, const int32_t* block_pairs, int num_pairs,
  * Supported: head_dim in {64, 128}; block_size in {16, 32}; num_q_heads a
  * multiple of num_kv_heads with group size 1..32 (above 8: the balanced
  * schedule only -- batch <= 4096, partition_tokens 0 or -1 -- and a
- * tensor-core variant; by default the tcgen05 consumer up to 16 columns,
+ * tensor-core variant; by default at head_dim 128 the tcgen05 consumer,
  * one CTA per SM streaming 128-token tiles).  Others: PA_ERR_UNSUPPORTED.
  * Launches: two kernels (decode + merge); the per-partition schedule skips
  * the merge when no request spans two partitions.
@@ -189,13 +189,13 @@ int pa_decode(pa_bf16* out, const pa_bf16* q, const pa_bf16* kv_pool,
 
 /* Kernel variant of the decode main loop. */
 typedef enum pa_decode_variant {
-  PA_DECODE_AUTO = 0,      /* 9..16 (token, head) columns per KV head: PA_DECODE_TCGEN05;
-                              otherwise PA_DECODE_MMA */
+  PA_DECODE_AUTO = 0,      /* 9..32 (token, head) columns per KV head at head_dim 128:
+                              PA_DECODE_TCGEN05; otherwise PA_DECODE_MMA */
   PA_DECODE_CUDA_CORE = 1, /* fp32 FMA on CUDA cores (group 1, 2 or 4) */
   PA_DECODE_MMA = 2,       /* bf16 mma.sync with fp32 accumulate (group 1..32) */
   PA_DECODE_TCGEN05 = 3    /* tcgen05.mma into tensor memory: 128-token tiles, one issuing
-                              thread, 1..16 columns; balanced schedule only (size the
-                              workspace with partition_tokens = -1) */
+                              thread, 1..32 columns (MMA N = 16 or 32); balanced schedule
+                              only (size the workspace with partition_tokens = -1) */
 } pa_decode_variant;
 
 /* pa_decode with explicit choices, for measurement and tests.
@@ -290,7 +290,8 @@ int pa_decode_append(pa_bf16* out, const pa_bf16* q, pa_bf16* kv_pool, const pa_
  *                pa_decode
  * Other arguments as pa_decode.  (num_q_heads / num_kv_heads) * T <= 32.
  * Always the balanced schedule (batch <= 4096) and a tensor-core consumer
- * (tcgen05 for 9..16 columns, mma.sync otherwise); workspace from
+ * (tcgen05 for 9..32 columns at head_dim 128, mma.sync otherwise);
+ * workspace from
  * pa_decode_multi_workspace_size.
  * ------------------------------------------------------------------------ */
 int pa_decode_multi_workspace_size(int batch, int num_query_tokens, int num_q_heads,

@@ -41,7 +41,7 @@ constexpr int kConsumerWarps = 4;
 constexpr int kThreads = (kConsumerWarps + 1) * 32;
 constexpr int kMaxGroup = 8;
 // The widest column count the default variant gives to the tcgen05 consumer.
-constexpr int kTcAutoMaxCols = 16;
+constexpr int kTcAutoMaxCols = 32;
 constexpr float kRescaleSlack = 8.f;  // log2 units: probabilities stay <= 256
 constexpr unsigned kFull = 0xffffffffu;
 
@@ -1486,9 +1486,11 @@ static int decode_impl(pa_bf16* out, const pa_bf16* q, const pa_bf16* kv_pool,
     return fail(PA_ERR_UNSUPPORTED, "multi-token decode has the tensor-core variants only");
   // tensor cores for every group: at scale mma.sync beats the CUDA-core
   // consumer even where the group leaves most of the 8-wide tile empty
-  // (g = 1, 2); from 9 to kTcAutoMaxCols columns the tcgen05 consumer takes over
+  // (g = 1, 2); from 9 to kTcAutoMaxCols columns of head dim 128 the tcgen05
+  // consumer takes over (at head dim 64 its 128-token tiles carry half the
+  // bytes for the same per-tile work, and mma.sync stays faster)
   if (variant == PA_DECODE_AUTO)
-    variant = (group * qtok > kMaxGroup && group * qtok <= kTcAutoMaxCols &&
+    variant = (group * qtok > kMaxGroup && group * qtok <= kTcAutoMaxCols && d == 128 &&
                tc_decode_supported(d, bs, group * qtok)) ? kTc : kMma;
   if (variant == kCudaCore && group != 1 && group != 2 && group != 4)
     return fail(PA_ERR_UNSUPPORTED, "pa_decode: CUDA-core variant has no group size %d", group);

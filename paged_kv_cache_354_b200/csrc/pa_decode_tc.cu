@@ -1,9 +1,11 @@
 // Balanced paged decode with a tcgen05 (tensor memory) consumer, for wide
 // column counts: GQA groups of 9..32 query heads per KV head, or several
 // query tokens per request (columns = query tokens x group, up to 32).
-// Columns come in halves of 16: every MMA has N = 16, every tensor-memory
-// access is 16 columns wide and every P tile 32 bytes wide; 17..32 columns
-// run two halves on each loaded tile.
+// Columns come in halves of 16: up to 16 columns one half, 17..32 two on
+// every loaded tile.  The MMAs cover all halves at once (N = 16 or 32);
+// every tensor-memory access is 16 columns wide and every P tile (one per
+// half) 32 bytes wide, the second reached through the descriptor's leading
+// byte offset.
 //
 // What it computes is pa_decode's (quiz page "PagedAttention (vLLM)", code
 // sketch "Conceptual: PagedAttention block lookup": keys and values of
@@ -19,11 +21,10 @@
 //    block as [8-row group][64-dim slab][row][64 dims] (128-byte swizzle), so
 //    in the tile the 8-token groups of every slab sit at one uniform stride
 //    and the tile is a canonical tensor-core operand;
-//  * one thread issues S^T = K Q^T (M = 128 tokens, N = 16 columns of a
-//    half, K = head dim) into tensor memory, then O^T += V^T P^T (M = head
-//    dim, N = the half's columns, K = the tile's tokens) into a
-//    tensor-memory accumulator per half that stays there for the whole
-//    (request, head) segment;
+//  * one thread issues S^T = K Q^T (M = 128 tokens, N = the columns held,
+//    K = head dim) into tensor memory, then O^T += V^T P^T (M = head dim,
+//    N = the columns held, K = the tile's tokens) into a tensor-memory
+//    accumulator that stays there for the whole (request, head) segment;
 //  * four softmax warps per half each own 32 token rows of S^T (one row per
 //    thread, the half's 16 columns in registers): mask, online max with a
 //    lagging kept max, probabilities rounded to bf16 into shared memory (the
@@ -65,7 +66,7 @@ constexpr int kTcRows = 128;         // M of S^T = K Q^T
 constexpr int kTcRingBytes = 196608; // K and V tiles in flight
 static_assert(kTcTileTokens % 32 == 0 && kTcTileTokens <= kTcRows, "tile of 32, 64, 96 or 128 tokens");
 constexpr float kTcSlack = 8.f;      // log2 units: probabilities stay <= 256
-constexpr int kTcHalf = 16;          // columns per MMA (N), per TMEM access, per P tile
+constexpr int kTcHalf = 16;          // columns per half: per TMEM access, per P tile, per softmax group
 constexpr int kTcMaxCols = 32;       // (token, head) columns per KV head: two halves
 
 template <int D, int BS, int NH>
@@ -420,11 +421,11 @@ __global__ void __launch_bounds__(tc_threads<NH>(), 1)
     } else if (warp == 1) {
       // --------------------------------------------------------- MMA issue
       if (lane == 0) {
-        constexpr uint32_t kIdS = tc::idesc_bf16(128, H16, false, false);
-        constexpr uint32_t kIdO = tc::idesc_bf16(128, H16, true, true);
+        constexpr uint32_t kIdSW = tc::idesc_bf16(128, NC, false, false);
+        constexpr uint32_t kIdOW = tc::idesc_bf16(128, NC, true, true);
         // S^T (tile i) = K Q^T over the head dim, 16 dims per instruction;
-        // half h2 multiplies Q rows [16 h2, 16 h2 + 16) (two 8-row groups
-        // further on) into its own 16 TMEM columns
+        // half h2's columns land in TMEM columns [16 h2, 16 h2 + 16) of the
+        // tile's buffer
         auto issue_s = [&](int i, const TileInfo& t) {
           const uint32_t kt = sbase + G::kK + (i % S) * G::kTileBytes;
           const uint32_t qt = sbase + G::kQ + (t.qseg & 1) * G::kQBytes;
@@ -433,17 +434,13 @@ __global__ void __launch_bounds__(tc_threads<NH>(), 1)
           for (int ks = 0; ks < D / 16; ++ks) {
             const int x = ks >> 2, kk = ks & 3;
             const uint64_t ad = tc::smem_desc(kt + x * 1024 + kk * 32, 16, G::kGroupStride, tc::kSwizzle128B);
-#pragma unroll
-            for (int h2 = 0; h2 < NH; ++h2) {
-              const uint64_t bd =
-                  tc::smem_desc(qt + x * G::kQSlab + h2 * 2048 + kk * 32, 16, 1024, tc::kSwizzle128B);
-              tc::mma_bf16(d + h2 * H16, ad, bd, kIdS, ks > 0 ? 1u : 0u);
-            }
+            // all NC rows of Q in one MMA of N = NC
+            const uint64_t bd = tc::smem_desc(qt + x * G::kQSlab + kk * 32, 16, 1024, tc::kSwizzle128B);
+            tc::mma_bf16(d, ad, bd, kIdSW, ks > 0 ? 1u : 0u);
           }
         };
-        // O^T += V^T P^T over the tile's real tokens, 16 per instruction, one
-        // accumulator per half; head dim 64 makes rows 64..127 repeat rows
-        // 0..63 (unused)
+        // O^T += V^T P^T over the tile's real tokens, 16 per instruction;
+        // head dim 64 makes rows 64..127 repeat rows 0..63 (unused)
         auto issue_pv = [&](int i, const TileInfo& t) {
           const uint32_t vt = sbase + G::kV + (i % S) * G::kTileBytes;
           const uint32_t pt = sbase + G::kP + (i & 1) * G::kPBytes;
@@ -451,12 +448,11 @@ __global__ void __launch_bounds__(tc_threads<NH>(), 1)
           for (int kk = 0; kk < steps; ++kk) {
             const uint64_t ad =
                 tc::smem_desc(vt + 2 * kk * G::kGroupStride, D == 128 ? 1024 : 0, G::kGroupStride, tc::kSwizzle128B);
-#pragma unroll
-            for (int h2 = 0; h2 < NH; ++h2) {
-              const uint64_t bd =
-                  tc::smem_desc(pt + h2 * G::kPHalf + kk * 16 * G::kPRow, 8192, 8 * G::kPRow, tc::kSwizzle32B);
-              tc::mma_bf16(tmem + 2 * NC + h2 * H16, ad, bd, kIdO, ((t.flags & kFirst) && kk == 0) ? 0u : 1u);
-            }
+            // both halves' P tiles in one MMA of N = NC: the second 16 columns
+            // sit one P tile further on (the leading byte offset)
+            const uint64_t bd = tc::smem_desc(pt + kk * 16 * G::kPRow, NH == 2 ? G::kPHalf : 8192, 8 * G::kPRow,
+                                              tc::kSwizzle32B);
+            tc::mma_bf16(tmem + 2 * NC, ad, bd, kIdOW, ((t.flags & kFirst) && kk == 0) ? 0u : 1u);
           }
         };
         auto give_up = [&]() {

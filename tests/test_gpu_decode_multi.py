@@ -43,8 +43,8 @@ def run_multi(q, pool, tables, lens, scale):
 
 
 # columns per KV head (group x T): 4, 16, 16, 16, 16, 9, 5, 12, 15, 32, 21,
-# 24, 32 -- 9 to 16 the tcgen05 consumer (one 16-column MMA tile), the rest
-# the mma.sync consumer
+# 24, 32 -- at head dim 128, 9 to 32 the tcgen05 consumer (one or two
+# 16-column halves); up to 8, and at head dim 64, the mma.sync consumer
 @pytest.mark.parametrize("T,hq,hkv", [(2, 8, 2), (4, 8, 2), (8, 4, 2), (2, 16, 2), (16, 2, 2), (3, 12, 4), (5, 4, 4),
                                       (3, 8, 2), (3, 10, 2), (4, 16, 2), (3, 14, 2), (3, 16, 2), (2, 32, 2)])
 @pytest.mark.parametrize("d,bs", [(128, 16), (64, 32), (64, 16)])
