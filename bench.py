@@ -300,11 +300,11 @@ def device_arm(name, K, W, rank, device, world, variant=0, partition_tokens=0, m
     """Device-timed figures of one workload, every input resident in HBM.
 
     Steps: W warm-up steps, then the same K steps (copy-on-write copies, the
-    fused cache write + decode + merge of one new token per request) repeated
-    R times so the timed region holds at least ``min_s`` of device time.
-    Decode alone: back-to-back pa_decode launches (main kernel + merge) on
-    the last step's inputs, repeated likewise.  Clocks are sampled over both
-    timed loops."""
+    fused cache write + decode + merge of one new token per request),
+    recorded once as a CUDA graph and replayed R times so the timed region
+    holds at least ``min_s`` of device time.  Decode alone: K back-to-back
+    pa_decode calls (main kernel + merge) on the last step's inputs, as a
+    graph replayed likewise.  Clocks are sampled over both timed loops."""
     import torch
     import torch.distributed as dist
 
@@ -330,15 +330,32 @@ def device_arm(name, K, W, rank, device, world, variant=0, partition_tokens=0, m
     def decode_once(i):
         cache.decode(qs[i % INPUT_SETS], out, d_tables[last], d_lens[last])
 
-    est_step = timed_ms(stream, lambda: [dev_step(i) for i in range(W)]) / W
-    est_dec = timed_ms(stream, lambda: [decode_once(i) for i in range(3)]) / 3
+    # W warm-up steps launched one by one, then the K timed steps (and K
+    # decode-only calls) recorded once as CUDA graphs: a replay runs every
+    # kernel of the K steps with no host launch work between them
+    for i in range(W):
+        dev_step(i)
+    for i in range(3):
+        decode_once(i)
+    torch.cuda.synchronize()
+
+    def record(fn):
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g):
+            fn()
+        return g
+
+    g_steps = record(lambda: [dev_step(i) for i in range(W, W + K)])
+    g_dec = record(lambda: [decode_once(i) for i in range(K)])
+    est_step = timed_ms(stream, g_steps.replay) / K
+    est_dec = timed_ms(stream, g_dec.replay) / K
     R = agree_max(repeats_for(est_step, K, min_s), device, world)
     Rd = agree_max(repeats_for(est_dec, K, min_s), device, world)
     if world > 1:
         dist.barrier()
     with ClockSampler(device.index) as clocks:
-        step_ms = timed_ms(stream, lambda: [dev_step(i) for _ in range(R) for i in range(W, W + K)])
-        dec_ms = timed_ms(stream, lambda: [decode_once(i) for i in range(Rd * K)])
+        step_ms = timed_ms(stream, lambda: [g_steps.replay() for _ in range(R)])
+        dec_ms = timed_ms(stream, lambda: [g_dec.replay() for _ in range(Rd)])
     if world > 1:
         dist.barrier()
     merge = 1 if (cache.schedule == "balanced" or cache.num_partitions > 1) else 0
@@ -529,8 +546,8 @@ def run_gpu(args):
             "data": "synthetic (seeded bf16 N(0,1) q/K/V; seeded lengths and shuffled block pool)",
             "config": workload_config(args.workload, steps_total(W, K), world),
             "run": {**summary, "timed_repeats": steps_timed // K, "steps_timed": steps_timed,
-                    "timing": "the K steps repeated timed_repeats times back to back (each repetition the same "
-                              "K steps: copy-on-write copies, fused cache write + decode + merge); one pair of "
+                    "timing": "the K steps (copy-on-write copies, fused cache write + decode + merge) recorded "
+                              "once as a CUDA graph and replayed timed_repeats times back to back; one pair of "
                               "CUDA events around all of them; ms_per_step = their device time / steps_timed"},
             "decode_seqs_per_s": round(batch * world * steps_timed / (step_ms * 1e-3), 1),
             "frac_of_hbm_peak": round(gbs / world / peaks["hbm_gbs"], 4),
