@@ -135,11 +135,42 @@ def test_tcgen05_matches_mma_sync(hq, hkv):
     assert (a.float() - b.float()).abs().max().item() <= 2 ** -7
 
 
-def test_balanced_schedule_at_its_batch_limit():
+@pytest.mark.parametrize("hq,variant", [(8, "mma"), (32, "tcgen05"), (64, "tcgen05")])
+def test_balanced_schedule_at_its_batch_limit(hq, variant):
     """4096 requests (the prefix table in shared memory at its largest) on the
-    balanced schedule, short ragged lengths including empty requests."""
+    balanced schedule, short ragged lengths including empty requests; the
+    tcgen05 consumer with one and with two halves.
+
+    With 0..39 positions an output averages a handful of value rows, so the
+    bf16 rounding of the probabilities (relative 2^-9 per weight, 2^-8 after
+    normalising) moves it by up to 2^-8 max_pos |v - out|, and the bf16
+    output by up to 2^-8 |out|; over the 0.5-1 M outputs of these shapes
+    that can pass 1e-2 with no kernel error at all.  Each element is bounded
+    by 1e-2 plus those two terms (the spread taken over the request's own
+    value rows); the mean stays <= 1e-3."""
     lens = list(np.random.default_rng(63).integers(0, 40, size=4096))
-    check(lens, 8, 2, 128, 16, seed=63, partition_tokens=pk.PA_SCHEDULE_BALANCED)
+    d, bs, hkv = 128, 16, 2
+    q, pool, (t_ref, l_ref), (t_cpp, l_cpp) = make_case(lens, hq, hkv, d, bs, seed=63)
+    scale = default_scale(d)
+    pool64, q64 = bf16_to_f64(pool), bf16_to_f64(q)
+    want = opa.decode(q64, pool64, t_ref, l_ref, scale)
+    out = run_decode(q.cuda(), pool.cuda(), t_cpp, l_cpp, scale, VARIANTS[variant], pk.PA_SCHEDULE_BALANCED)
+    assert pk.pa_device_error() == 0
+    got = bf16_to_f64(out)
+    g = hq // hkv
+    spread = np.zeros_like(want)
+    for b, n in enumerate(l_ref):
+        if n == 0:
+            continue
+        rows = np.stack([pool64[t_ref[b][p // bs], 1, :, p % bs, :] for p in range(int(n))])  # [n, hkv, d]
+        vmax = np.repeat(rows.max(axis=0), g, axis=0)  # [hq, d]: query head j reads KV head j // g
+        vmin = np.repeat(rows.min(axis=0), g, axis=0)
+        spread[b] = np.maximum(np.abs(vmax - want[b]), np.abs(vmin - want[b]))
+    err = np.abs(got - want)
+    assert np.isfinite(got).all()
+    bound = 1e-2 + 2.0 ** -8 * (spread + np.abs(want))
+    assert (err <= bound).all(), float((err - bound).max())
+    assert err.mean() <= 1e-3
 
 
 def test_batch_above_balanced_limit_uses_grid():
