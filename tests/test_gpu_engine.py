@@ -95,8 +95,8 @@ def test_graph_replayed_steps_match_oracle(schedule):
     assert pk.pa_device_error() == 0
 
 
-@pytest.mark.parametrize("zero_copy", [True, False])
-def test_whole_step_graphs_match_oracle(zero_copy):
+@pytest.mark.parametrize("zero_copy,hq", [(True, 8), (False, 8), (True, 32), (True, 48)])
+def test_whole_step_graphs_match_oracle(zero_copy, hq):
     """capture_steps: upload and fused decode as one graph per staging
     buffer, the output reaching pinned host memory straight from the kernels
     (zero_copy) or through a device-to-host copy in the graph (steps with
@@ -104,7 +104,7 @@ def test_whole_step_graphs_match_oracle(zero_copy):
     output equals the oracle's replay, and the pool equals the oracle's bit
     for bit."""
     dev = torch.device("cuda", torch.cuda.current_device())
-    hq, hkv, d, bs, sets = 8, 2, 128, 16, 3
+    hkv, d, bs, sets = 2, 128, 16, 3  # hq 32 / 48: groups 16 / 24 on the tcgen05 consumer
     nb = 200
     order = np.random.default_rng(11).permutation(nb)
     cache = PagedDecodeCache(nb, hq, hkv, d, bs, max_batch=4, max_seq_len=700, initial_order=order,
