@@ -1565,10 +1565,11 @@ static int decode_impl(pa_bf16* out, const pa_bf16* q, const pa_bf16* kv_pool,
   a.seg_extra = tc ? tc_decode_segment_extra(bs) : (plan.stream ? kStreamSegExtraTokens / stream_tile(d, bs) : 0);
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   if (fused) {
-    // the decode kernel patches the staged tile, the merge kernel stores the
-    // row; with block pairs, paired warps or the tcgen05 consumer the cache
+    // mma.sync: the decode kernel patches the staged tile, the merge kernel
+    // stores the row; tcgen05: the decode kernel stores the row before the
+    // TMA load of its block; with block pairs or paired warps the cache
     // write runs first
-    if (plan.stream && !pairs && !tc && a.cols <= kMaxGroup) {
+    if (plan.stream && !pairs && (tc || a.cols <= kMaxGroup)) {
       a.new_k = reinterpret_cast<const uint4*>(new_k);
       a.new_v = reinterpret_cast<const uint4*>(new_v);
       a.new_slots = new_slots;

@@ -37,7 +37,7 @@ struct DecodeArgs {
   const uint4* new_k;
   const uint4* new_v;
   const int64_t* new_slots;
-  uint4* pool_w;       // the pool, written by the merge kernel
+  uint4* pool_w;       // the pool, for the fused cache write (merge kernel, or the tcgen05 decode kernel)
   // balanced schedule: virtual work units added to every (request, KV head)
   // that has blocks, so a CTA covering many short ones takes fewer real
   // blocks (per-segment costs); they carry no data and are skipped

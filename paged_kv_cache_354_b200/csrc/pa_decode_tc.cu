@@ -189,6 +189,21 @@ __device__ __forceinline__ float warp_columns(float (&v)[kTcHalf], int lane) {
   return v[0];
 }
 
+// Fused cache write: part p of request b's newest key / value row of KV
+// head h (p < D/8: 16 bytes of the key, else of the value) into its slot of
+// the pool.  A slot past the pool is flagged and skipped.
+template <int D, int BS>
+__device__ __forceinline__ void store_new_part(const DecodeArgs& a, long long slot, int b, int h, int p,
+                                               uint4 v) {
+  if (slot >= static_cast<long long>(a.num_blocks) * BS) {
+    flag_error(a.err, PA_DEVERR_SLOT);
+    return;
+  }
+  const int kv = p / (D / 8), chunk = p % (D / 8);
+  const long long blk = slot / BS, off = slot - blk * BS;
+  a.pool_w[(((blk * 2 + kv) * a.num_kv_heads + h) * BS + off) * (D / 8) + chunk] = v;
+}
+
 template <int D, int BS, int NH>
 __global__ void __launch_bounds__(tc_threads<NH>(), 1)
     paged_decode_tc_kernel(const __grid_constant__ CUtensorMap kv_map, const __grid_constant__ CUtensorMap q_map,
@@ -292,6 +307,19 @@ __global__ void __launch_bounds__(tc_threads<NH>(), 1)
     }
     v -= kk - nreal + 1;  // the last real block of this (b, h)
   }
+  // fused cache write for requests with no block to attend over: no CTA's
+  // range holds them, so CTA 0 stores their rows (nothing reads them here)
+  if (a.new_k != nullptr && blockIdx.x == 0) {
+    for (int b = threadIdx.x; b < batch; b += kThreads) {
+      const long long slot = prefix[b + 1] == prefix[b] ? __ldg(a.new_slots + b) : -1;
+      if (slot < 0) continue;
+      for (int h = 0; h < hkv; ++h)
+        for (int p = 0; p < 2 * (D / 8); ++p) {
+          const uint4* src = (p < D / 8 ? a.new_k : a.new_v) + (static_cast<size_t>(b) * hkv + h) * (D / 8) + p % (D / 8);
+          store_new_part<D, BS>(a, slot, b, h, p, __ldg(src));
+        }
+    }
+  }
   fence_proxy_async_smem();  // the ring's generic writes above, TMA writes below
   tc::fence_before_sync();
   __syncthreads();
@@ -338,6 +366,16 @@ __global__ void __launch_bounds__(tc_threads<NH>(), 1)
           }
           break;
         }
+        // fused cache write: the CTA that streams this (b, h)'s last block
+        // stores the newest token's key and value rows into their slot just
+        // before that block's TMA load (only this CTA reads the block's rows
+        // of head h); lane p fetches part p now
+        const bool writes_new = a.new_k != nullptr && k + cnt == nb;
+        const long long new_slot = writes_new ? __ldg(a.new_slots + b) : -1;
+        uint4 new_part = make_uint4(0u, 0u, 0u, 0u);
+        if (new_slot >= 0 && lane < 2 * (D / 8))
+          new_part = __ldg((lane < D / 8 ? a.new_k : a.new_v) + (static_cast<size_t>(b) * hkv + h) * (D / 8) +
+                           lane % (D / 8));
         const int32_t* trow = a.block_tables + static_cast<size_t>(b) * a.max_blocks_per_seq + k;
         for (int base = 0; base < cnt && !stop; base += G::kChunk) {
           int phys = 0;
@@ -354,6 +392,13 @@ __global__ void __launch_bounds__(tc_threads<NH>(), 1)
             int pb[G::kTileBlocks];
 #pragma unroll
             for (int j = 0; j < G::kTileBlocks; ++j) pb[j] = __shfl_sync(kFullMask, phys, (t0 + j) & 31);
+            if (new_slot >= 0 && base + t0 + nblk == cnt) {  // the tile with the last block
+              if (lane < 2 * (D / 8)) {
+                store_new_part<D, BS>(a, new_slot, b, h, lane, new_part);
+                fence_proxy_async_global();  // before lane 0's TMA load of the block
+              }
+              __syncwarp();
+            }
             failed = 0;
             if (lane == 0) {
               const int s = i % S;
@@ -798,7 +843,10 @@ int launch_tc_decode(const DecodeArgs& a, const void* kv_pool, int batch, int d,
   else rc = bs == 16 ? launch_tc_cols<64, 16>(kv_map, q_map, a, batch, ctas, st)
                      : launch_tc_cols<64, 32>(kv_map, q_map, a, batch, ctas, st);
   if (rc != PA_OK) return rc;
-  return launch_stream_merge(d, bs, a, batch, ctas, st);
+  DecodeArgs m = a;
+  m.new_k = m.new_v = nullptr;  // the decode kernel stored the new rows already
+  m.new_slots = nullptr;
+  return launch_stream_merge(d, bs, m, batch, ctas, st);
 }
 
 }  // namespace pa

@@ -27,7 +27,10 @@ def bits(t):
     ([900, 33, 5, 2047, 400], 16, 4, 64, 32),                      # balanced, other shape
     ([3, 20, 1], 4, 4, 64, 16),                                    # little work: per-partition grid
     ([900, 33, 5, 2047, 400, 1600, 2500, 3000], 16, 4, 64, 16),   # balanced on block pairs: write, then decode
-    ([700, 1, 2049, 64, 300, 1500, 17, 1024], 32, 2, 128, 16),    # group 16 (paired warps): write, then decode
+    ([700, 1, 2049, 64, 300, 1500, 17, 1024], 32, 2, 128, 16),    # group 16 (tcgen05): stored before the TMA load
+    ([700, 1, 2049, 64, 300, 1500, 17, 1024], 48, 2, 128, 32),    # group 24 (tcgen05, two halves), bs32
+    ([900, 33, 5, 2047, 400, 128, 127, 129], 64, 4, 128, 16),     # group 16, tile edges
+    ([700, 1, 2049, 64, 300, 1500, 17, 1024], 32, 2, 64, 16),     # group 16 at head dim 64 (paired warps): write, then decode
 ])
 def test_append_equals_separate_calls(lens, hq, hkv, d, bs):
     dev = torch.device("cuda", torch.cuda.current_device())
@@ -77,9 +80,13 @@ def test_append_equals_separate_calls(lens, hq, hkv, d, bs):
     compare(out_b.double().cpu().numpy(), want)
 
 
-def test_append_with_empty_requests():
+@pytest.mark.parametrize("hq", [8, 32])
+def test_append_with_empty_requests(hq):
+    """Empty requests with and without a slot (one writes into a block no
+    request holds: only the cache write touches it); group 4 on mma.sync,
+    group 16 on the tcgen05 consumer."""
     dev = torch.device("cuda", torch.cuda.current_device())
-    hq, hkv, d, bs = 8, 2, 128, 16
+    hkv, d, bs = 2, 128, 16
     lens = [0, 1500, 0, 2000] * 8  # 32 requests, enough work for the balanced schedule
     nb = sum(-(-n // bs) for n in lens) + 4
     a = pk.PaAlloc(nb, bs)
@@ -92,6 +99,7 @@ def test_append_with_empty_requests():
     slots_live, _ = a.append_batch(live, 1, as_numpy=True)
     slots = np.full(len(lens), -1, dtype=np.int64)
     slots[live] = slots_live
+    slots[2] = (nb - 1) * bs + 3  # an empty request with a slot, in the last (free) block
     tables, l = a.block_tables(ids, max(-(-n // bs) for n in lens))
     assert list(l) == lens
     pool = workloads.bf16_normal((nb, 2, hkv, bs, d), seed=7).to(dev)
