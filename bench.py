@@ -169,6 +169,31 @@ def l2_note(plan_step, kv_logical, cache):
             f"not a bandwidth measurement")
 
 
+def workload_l2(p):
+    """Whether the workload's K/V of one step exceeds the L2 (no flush is
+    used between steps): from its tables as the decode steps start (the
+    beams' divergent tokens appended), so both arms print the same
+    statement."""
+    from paged_kv_cache_354_b200 import PaAlloc
+
+    s = p.shape
+    alloc = PaAlloc(p.num_blocks, s.block_size, p.initial_order)
+    ids = workloads.populate(alloc, p)
+    if p.name == "beam":
+        alloc.append_batch(ids, p.append_tokens)
+    tables, lens = workloads.block_tables(alloc, ids)
+    nblk = -(-np.asarray(lens, dtype=np.int64) // s.block_size)
+    per_block = 2 * s.num_kv_heads * s.block_size * s.head_dim * 2
+    logical = int(nblk.sum()) * per_block
+    distinct = len(np.unique(np.concatenate([t[:n] for t, n in zip(tables, nblk)]))) * per_block
+    if distinct > L2_BYTES:
+        return f"inputs larger than L2 ({distinct / 1e6:.0f} MB of K/V blocks > 126 MB), no flush"
+    if logical > L2_BYTES:
+        return (f"{logical / 1e6:.0f} MB of K/V read per step from {distinct / 1e6:.0f} MB of shared blocks "
+                f"(L2 126 MB), no flush: shared blocks may come from L2")
+    return f"inputs fit in L2 ({logical / 1e6:.1f} MB), no flush: launch-bound, not a bandwidth measurement"
+
+
 def workload_config(name, steps_total, world):
     """The workload fields of the JSON line's ``config``, shared by both arms."""
     p = workloads.plan(name, extra_tokens=steps_total + 1)
@@ -179,6 +204,7 @@ def workload_config(name, steps_total, world):
         "batch": batch, "num_q_heads": s.num_q_heads, "num_kv_heads": s.num_kv_heads, "head_dim": s.head_dim,
         "block_size": s.block_size, "num_blocks": p.num_blocks,
         "parallelism": f"dp{world} (independent batches, no collective)",
+        "l2": workload_l2(p),
     }
 
 
