@@ -169,9 +169,11 @@ int pa_copy_blocks(pa_bf16* kv_pool, const int32_t* block_pairs, int num_pairs,
  * tokens) and the same kind of merge.
  * Supported: head_dim in {64, 128}; block_size in {16, 32}; num_q_heads a
  * multiple of num_kv_heads with group size 1..32 (above 8: the balanced
- * schedule only -- batch <= 4096, partition_tokens 0 or -1 -- and a
- * tensor-core variant; by default at head_dim 128 the tcgen05 consumer,
- * one CTA per SM streaming 128-token tiles).  Others: PA_ERR_UNSUPPORTED.
+ * schedule only -- partition_tokens 0 or -1 -- and a tensor-core variant;
+ * by default at head_dim 128 the tcgen05 consumer, one CTA per SM
+ * streaming 128-token tiles; batches of 4097..32768 requests run on the
+ * tcgen05 consumer at either head_dim, up to 4096 on either).  Others:
+ * PA_ERR_UNSUPPORTED.
  * Launches: two kernels (decode + merge); the per-partition schedule skips
  * the merge when no request spans two partitions.
  * ------------------------------------------------------------------------ */
@@ -293,7 +295,8 @@ int pa_decode_append(pa_bf16* out, const pa_bf16* q, pa_bf16* kv_pool, const pa_
  *                memory, out in device or pinned host memory as for
  *                pa_decode
  * Other arguments as pa_decode.  (num_q_heads / num_kv_heads) * T <= 32.
- * Always the balanced schedule (batch <= 4096) and a tensor-core consumer
+ * Always the balanced schedule (batch <= 4096; above 8 columns up to
+ * 32768 requests, on the tcgen05 consumer) and a tensor-core consumer
  * (tcgen05 for 9..32 columns at head_dim 128, mma.sync otherwise);
  * workspace from
  * pa_decode_multi_workspace_size.

@@ -721,6 +721,10 @@ constexpr int kStreamCtasPerSm = PA_STREAM_CTAS_PER_SM;
 #endif
 constexpr int kStreamSegExtraTokens = PA_STREAM_SEG_EXTRA_TOKENS;
 constexpr int kStreamMaxBatch = 4096;  // the prefix table lives in shared memory
+// The tcgen05 consumer builds its prefix table in its idle tile ring at the
+// start, so it takes larger batches: more than 8 columns above
+// kStreamMaxBatch requests run there whatever the head dim.
+constexpr int kTcMaxBatch = 32768;
 
 // Consumer groups of the balanced kernel: with up to 8 (token, head) columns
 // each consumer warp takes every fourth block alone; with up to 16 (two
@@ -1296,7 +1300,10 @@ static int make_plan(int batch, int hq, int hkv, int d, int bs, int max_seq_len,
   const int tile = stream_tile(d, bs);
   const long long units_max =
       static_cast<long long>(batch) * hkv * (max_seq_len > 0 ? (max_seq_len + tile - 1) / tile : 1);
-  if (partition_tokens == kForceBalanced && batch > kStreamMaxBatch)
+  const bool tc_only = group * qtok > kMaxGroup && batch > kStreamMaxBatch;  // only the tcgen05 consumer fits
+  if (tc_only && (batch > kTcMaxBatch || !tc_decode_supported(d, bs, group * qtok)))
+    return fail(PA_ERR_UNSUPPORTED, "balanced schedule: batch %d above %d", batch, kTcMaxBatch);
+  if (partition_tokens == kForceBalanced && batch > kStreamMaxBatch && !tc_only)
     return fail(PA_ERR_UNSUPPORTED, "balanced schedule: batch %d above %d", batch, kStreamMaxBatch);
   if (partition_tokens == kForceBalanced ||
       (partition_tokens == 0 && batch <= kStreamMaxBatch &&
@@ -1490,8 +1497,11 @@ static int decode_impl(pa_bf16* out, const pa_bf16* q, const pa_bf16* kv_pool,
   // consumer takes over (at head dim 64 its 128-token tiles carry half the
   // bytes for the same per-tile work, and mma.sync stays faster)
   if (variant == PA_DECODE_AUTO)
-    variant = (group * qtok > kMaxGroup && group * qtok <= kTcAutoMaxCols && d == 128 &&
-               tc_decode_supported(d, bs, group * qtok)) ? kTc : kMma;
+    variant = (group * qtok > kMaxGroup && group * qtok <= kTcAutoMaxCols &&
+               (d == 128 || batch > kStreamMaxBatch) && tc_decode_supported(d, bs, group * qtok)) ? kTc : kMma;
+  if (group * qtok > kMaxGroup && batch > kStreamMaxBatch && variant != kTc)
+    return fail(PA_ERR_UNSUPPORTED, "pa_decode: more than %d columns with batch %d above %d: the tcgen05 variant only",
+                kMaxGroup, batch, kStreamMaxBatch);
   if (variant == kCudaCore && group != 1 && group != 2 && group != 4)
     return fail(PA_ERR_UNSUPPORTED, "pa_decode: CUDA-core variant has no group size %d", group);
   if (variant != kCudaCore && variant != kMma && variant != kTc)

@@ -809,6 +809,9 @@ int launch_tc_decode(const DecodeArgs& a, const void* kv_pool, int batch, int d,
                      cudaStream_t st) {
   if (!tc_decode_supported(d, bs, a.cols))
     return fail(PA_ERR_UNSUPPORTED, "tcgen05 decode: head_dim %d, block_size %d, %d columns", d, bs, a.cols);
+  // the prefix table and its scan scratch are built in the (still idle) tile ring
+  if (((batch + 1 + 3) & ~3) + tc_threads<2>() + 1 > kTcRingBytes / 4)
+    return fail(PA_ERR_UNSUPPORTED, "tcgen05 decode: batch %d too large for the prefix table", batch);
   const int hkv = a.num_kv_heads;
   const int hq = a.num_q_heads;
   // Pool view, 5-D: x = dim within a 64-dim slab, y = row within an 8-row

@@ -66,7 +66,10 @@ def test_invalid_arguments_fail_before_launch():
     # groups above 8 run on the balanced schedule only
     assert lib.pa_decode_workspace_size_ex(4, 32, 2, 128, 16, 1000, 256, ctypes.byref(nb),
                                            ctypes.byref(parts), None) == pk.PA_ERR_UNSUPPORTED
+    # ... and above 4096 requests on the tcgen05 consumer only, up to 32768
     assert lib.pa_decode_workspace_size_ex(5000, 32, 2, 128, 16, 1000, 0, ctypes.byref(nb),
+                                           ctypes.byref(parts), None) == pk.PA_OK
+    assert lib.pa_decode_workspace_size_ex(40000, 32, 2, 128, 16, 1000, 0, ctypes.byref(nb),
                                            ctypes.byref(parts), None) == pk.PA_ERR_UNSUPPORTED
     assert lib.pa_decode_workspace_size(4, 6, 4, 128, 16, 100, ctypes.byref(nb), ctypes.byref(parts)) == \
         pk.PA_ERR_INVALID

@@ -135,26 +135,20 @@ def test_tcgen05_matches_mma_sync(hq, hkv):
     assert (a.float() - b.float()).abs().max().item() <= 2 ** -7
 
 
-@pytest.mark.parametrize("hq,variant", [(8, "mma"), (32, "tcgen05"), (64, "tcgen05")])
-def test_balanced_schedule_at_its_batch_limit(hq, variant):
-    """4096 requests (the prefix table in shared memory at its largest) on the
-    balanced schedule, short ragged lengths including empty requests; the
-    tcgen05 consumer with one and with two halves.
-
-    With 0..39 positions an output averages a handful of value rows, so the
-    bf16 rounding of the probabilities (relative 2^-9 per weight, 2^-8 after
-    normalising) moves it by up to 2^-8 max_pos |v - out|, and the bf16
-    output by up to 2^-8 |out|; over the 0.5-1 M outputs of these shapes
-    that can pass 1e-2 with no kernel error at all.  Each element is bounded
-    by 1e-2 plus those two terms (the spread taken over the request's own
-    value rows); the mean stays <= 1e-3."""
-    lens = list(np.random.default_rng(63).integers(0, 40, size=4096))
-    d, bs, hkv = 128, 16, 2
-    q, pool, (t_ref, l_ref), (t_cpp, l_cpp) = make_case(lens, hq, hkv, d, bs, seed=63)
+def check_short(lens, hq, hkv, d, bs, seed, variant="auto", partition_tokens=pk.PA_SCHEDULE_BALANCED):
+    """check() for batches of very short requests (0..~40 positions): an
+    output then averages a handful of value rows, so the bf16 rounding of the
+    probabilities (relative 2^-9 per weight, 2^-8 after normalising) moves it
+    by up to 2^-8 max_pos |v - out|, and the bf16 output by up to 2^-8
+    |out|; over the 0.5-1 M outputs of these shapes that can pass 1e-2 with
+    no kernel error at all.  Each element is bounded by 1e-2 plus those two
+    terms (the spread over the request's own value rows); the mean stays
+    <= 1e-3."""
+    q, pool, (t_ref, l_ref), (t_cpp, l_cpp) = make_case(lens, hq, hkv, d, bs, seed=seed)
     scale = default_scale(d)
     pool64, q64 = bf16_to_f64(pool), bf16_to_f64(q)
     want = opa.decode(q64, pool64, t_ref, l_ref, scale)
-    out = run_decode(q.cuda(), pool.cuda(), t_cpp, l_cpp, scale, VARIANTS[variant], pk.PA_SCHEDULE_BALANCED)
+    out = run_decode(q.cuda(), pool.cuda(), t_cpp, l_cpp, scale, VARIANTS[variant], partition_tokens)
     assert pk.pa_device_error() == 0
     got = bf16_to_f64(out)
     g = hq // hkv
@@ -171,6 +165,27 @@ def test_balanced_schedule_at_its_batch_limit(hq, variant):
     bound = 1e-2 + 2.0 ** -8 * (spread + np.abs(want))
     assert (err <= bound).all(), float((err - bound).max())
     assert err.mean() <= 1e-3
+
+
+@pytest.mark.parametrize("hq,variant", [(8, "mma"), (32, "tcgen05"), (64, "tcgen05")])
+def test_balanced_schedule_at_its_batch_limit(hq, variant):
+    """4096 requests (the prefix table in shared memory at its largest) on the
+    balanced schedule, short ragged lengths including empty requests; the
+    tcgen05 consumer with one and with two halves."""
+    lens = list(np.random.default_rng(63).integers(0, 40, size=4096))
+    check_short(lens, hq, 2, 128, 16, seed=63, variant=variant)
+
+
+@pytest.mark.parametrize("hq,d,bs", [(32, 128, 16), (32, 64, 16), (48, 128, 32)])
+def test_wide_groups_above_the_batch_limit(hq, d, bs):
+    """More than 8 columns with more than 4096 requests: the default variant
+    runs the tcgen05 consumer (its prefix table lives in the tile ring), at
+    head dim 64 too; mma.sync is refused."""
+    lens = list(np.random.default_rng(64).integers(0, 30, size=4200))
+    check_short(lens, hq, 2, d, bs, seed=64, variant="auto", partition_tokens=0)
+    q, pool, _, (t, l) = make_case(lens[:4200], hq, 2, d, bs, seed=65)
+    with pytest.raises(pk.PaError):
+        run_decode(q.cuda(), pool.cuda(), t, l, 0.1, pk.PA_DECODE_MMA, pk.PA_SCHEDULE_BALANCED)
 
 
 def test_batch_above_balanced_limit_uses_grid():

@@ -31,6 +31,7 @@ def bits(t):
     ([700, 1, 2049, 64, 300, 1500, 17, 1024], 48, 2, 128, 32),    # group 24 (tcgen05, two halves), bs32
     ([900, 33, 5, 2047, 400, 128, 127, 129], 64, 4, 128, 16),     # group 16, tile edges
     ([700, 1, 2049, 64, 300, 1500, 17, 1024], 32, 2, 64, 16),     # group 16 at head dim 64 (paired warps): write, then decode
+    ([int(x) for x in np.random.default_rng(67).integers(1, 30, size=4200)], 32, 2, 64, 16),  # 4200 requests: tcgen05
 ])
 def test_append_equals_separate_calls(lens, hq, hkv, d, bs):
     dev = torch.device("cuda", torch.cuda.current_device())
@@ -77,7 +78,14 @@ def test_append_equals_separate_calls(lens, hq, hkv, d, bs):
     assert np.array_equal(bits(pool_b), want_pool)
     t_ref, l_ref = workloads.block_tables(ref, ids, mb)
     want = opa.decode(q.double().cpu().numpy(), u16_to_f64(want_pool), t_ref, l_ref, scale)
-    compare(out_b.double().cpu().numpy(), want)
+    if len(lens) <= 4096:
+        compare(out_b.double().cpu().numpy(), want)
+    else:
+        # thousands of requests of a few positions: the bf16 probabilities and
+        # output can move an element by 2^-8 (|v - out| spread + |out|) beyond
+        # 1e-2 (tests/test_gpu_decode.py, check_short); |v| < ~5.5 here
+        err = np.abs(out_b.double().cpu().numpy() - want)
+        assert err.mean() <= 1e-3 and (err <= 1e-2 + 2.0 ** -8 * (11.0 + np.abs(want))).all()
 
 
 @pytest.mark.parametrize("hq", [8, 32])

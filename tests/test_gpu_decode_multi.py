@@ -80,3 +80,21 @@ def test_single_token_matches_pa_decode():
 def test_multi_rejects_too_wide_tiles():
     with pytest.raises(pk.PaError):
         pk.pa_decode_multi_workspace_size(4, 3, 96, 8, 128, 16, 100)  # group 12 x 3 tokens = 36 columns
+
+
+def test_multi_above_the_batch_limit():
+    """4200 requests, 2 query tokens x group 8 (16 columns): the tcgen05
+    consumer, whose prefix table takes batches above 4096."""
+    lens = [int(x) for x in np.random.default_rng(66).integers(0, 24, size=4200)]
+    T, hq, hkv, d, bs = 2, 16, 2, 128, 16
+    q, pool, (t_ref, l_ref), (t, l) = make(lens, T, hq, hkv, d, bs, seed=66)
+    scale = 1.0 / math.sqrt(d)
+    want = opa.decode_multi(bf16_to_f64(q), bf16_to_f64(pool), t_ref, l_ref, scale)
+    got = bf16_to_f64(run_multi(q.cuda(), pool.cuda(), t, l, scale))
+    assert pk.pa_device_error() == 0
+    # very short requests: the bf16 probabilities and output can move an
+    # element by 2^-8 (|v - out| spread + |out|) beyond the 1e-2 bound (see
+    # tests/test_gpu_decode.py, check_short); with |v| < ~5.5 that is < 0.065
+    err = np.abs(got - want)
+    assert np.isfinite(got).all() and err.mean() <= 1e-3
+    assert (err <= 1e-2 + 2.0 ** -8 * (11.0 + np.abs(want))).all()
