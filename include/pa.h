@@ -330,7 +330,8 @@ int pa_decode_multi(pa_bf16* out, const pa_bf16* q, const pa_bf16* kv_pool,
  * max_len must be a positive multiple of 16; seq_lens[b] > max_len is
  * flagged (PA_DEVERR_SEQ_LEN) and clamped.  variant: PA_DECODE_AUTO,
  * PA_DECODE_CUDA_CORE (group 1, 2, 4) or PA_DECODE_MMA.  batch <= 4096,
- * group <= 8.
+ * group <= 32 (above 8: mma.sync on grouped warps, as pa_decode with
+ * PA_DECODE_MMA on the balanced schedule).
  * Workspace from pa_decode_contiguous_workspace_size (never 0 bytes).
  * Other arguments as pa_decode (out in device or pinned host memory).
  * ------------------------------------------------------------------------ */

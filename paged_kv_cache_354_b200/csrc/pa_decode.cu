@@ -1607,6 +1607,8 @@ template <int D>
 static int dispatch_contiguous(const CUtensorMap& map, const DecodeArgs& a, int batch, int variant,
                                int ctas, cudaStream_t st) {
   constexpr int T = kContiguousTile;
+  if (variant == kMma && a.cols > 16) return launch_stream<D, T, kMma, 0, 4, kContiguous>(map, a, batch, ctas, st);
+  if (variant == kMma && a.cols > 8) return launch_stream<D, T, kMma, 0, 2, kContiguous>(map, a, batch, ctas, st);
   if (variant == kMma) return launch_stream<D, T, kMma, 0, 1, kContiguous>(map, a, batch, ctas, st);
   switch (a.group) {
     case 1: return launch_stream<D, T, kCudaCore, 1, 1, kContiguous>(map, a, batch, ctas, st);
@@ -1623,8 +1625,12 @@ static int contiguous_plan(int batch, int hq, int hkv, int d, int max_len, Plan*
   if (max_len <= 0 || max_len % kContiguousTile != 0)
     return fail(PA_ERR_INVALID, "pa_decode_contiguous: max_len %d not a positive multiple of %d", max_len,
                 kContiguousTile);
-  if (hq / hkv > kMaxGroup)
-    return fail(PA_ERR_UNSUPPORTED, "pa_decode_contiguous: group size %d above %d", hq / hkv, kMaxGroup);
+  if (hq / hkv > 4 * kMaxGroup)
+    return fail(PA_ERR_UNSUPPORTED, "pa_decode_contiguous: group size %d above %d", hq / hkv, 4 * kMaxGroup);
+  if (batch > kStreamMaxBatch)
+    return fail(PA_ERR_UNSUPPORTED, "pa_decode_contiguous: batch %d above %d", batch, kStreamMaxBatch);
+  // (above 8 query heads per KV head: the mma.sync kernel's grouped warps,
+  // as pa_decode on request, so the two layouts still compare kernel for kernel)
   return make_plan(batch, hq, hkv, d, kContiguousTile, max_len, kForceBalanced, plan);
 }
 

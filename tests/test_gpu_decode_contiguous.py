@@ -59,7 +59,8 @@ RAGGED = [1, 15, 16, 17, 32, 53, 100, 257, 600, 0]
 
 @pytest.mark.parametrize("d", [64, 128])
 @pytest.mark.parametrize("variant,group", [("auto", 1), ("auto", 2), ("auto", 4), ("auto", 8),
-                                           ("cuda_core", 4), ("mma", 1), ("mma", 3)])
+                                           ("cuda_core", 4), ("mma", 1), ("mma", 3),
+                                           ("auto", 16), ("mma", 12), ("mma", 24), ("auto", 32)])
 def test_parity_with_oracle(d, variant, group):
     hkv, max_len = 2, 608
     cache = make_cache(RAGGED, hkv, d, max_len, seed=31 + group + d)
@@ -71,11 +72,12 @@ def test_parity_with_oracle(d, variant, group):
     compare(bf16_to_f64(out), want)
 
 
-@pytest.mark.parametrize("variant", ["auto", "cuda_core", "mma"])
+@pytest.mark.parametrize("variant,group", [("auto", 4), ("cuda_core", 4), ("mma", 4), ("mma", 16), ("mma", 32)])
 @pytest.mark.parametrize("lens", [RAGGED, [40000], [3, 0, 1]])
-def test_bitwise_equal_to_paged(variant, lens):
-    """Same lengths -> same units, same CTA ranges, same arithmetic."""
-    hkv, group, d = 2, 4, 128
+def test_bitwise_equal_to_paged(variant, group, lens):
+    """Same lengths -> same units, same CTA ranges, same arithmetic (groups
+    16 and 32: the grouped-warp mma.sync kernel in both layouts)."""
+    hkv, d = 2, 128
     max_len = -(-max(lens) // 16) * 16 + 16
     cache = make_cache(lens, hkv, d, max_len, seed=41)
     q = workloads.bf16_normal((len(lens), hkv * group, d), seed=42)
