@@ -263,12 +263,12 @@ int pa_decode_noalloc(pa_bf16* out, const pa_bf16* q, const pa_bf16* kv_pool,
  * that position's slot (block_tables[b][(L-1)/bs] * bs + (L-1) % bs, as
  * pa_alloc_append returns it); a negative slot writes nothing.  On the
  * balanced schedule there is no separate cache-write launch: the mma.sync
- * decode kernel puts the new row straight into the staged tile and the merge
- * kernel stores it in the pool afterwards; the tcgen05 one stores it in the
- * pool just before loading that block (the only CTA that reads those rows).
- * With block pairs (head_dim 64, block_size 16) or paired warps (more than 8
- * columns at head_dim 64), and on the per-partition grid, the two kernels
- * run in turn.
+ * decode kernel with one warp per block puts the new row straight into the
+ * staged tile and the merge kernel stores it in the pool afterwards; the
+ * tcgen05 kernel, the grouped-warp and the block-pair mma.sync kernels
+ * store it in the pool just before the TMA load of that block (their CTA is
+ * the only one that reads those rows).  On the per-partition grid the two
+ * kernels run in turn.
  * new_k, new_v : device bf16 [batch][num_kv_heads][head_dim]
  * slot_mapping : device int64 [batch]
  * Other arguments, workspace and limits as pa_decode.

@@ -828,6 +828,13 @@ __global__ void __launch_bounds__(kThreads, kStreamCtasPerSm)
   const long long total = static_cast<long long>(hkv) * prefix[batch];
   const long long u_begin = stream_begin(total, blockIdx.x, ctas);
   const long long u_end = stream_begin(total, blockIdx.x + 1, ctas);
+  // fused cache write where the consumers cannot patch the staged tile (warp
+  // groups share it; a block-pair tile holds two blocks): the producer
+  // stores the newest row into its slot just before the TMA load of the
+  // (b, h)'s last tile, and CTA 0 stores the rows of requests with no block
+  constexpr bool kStoreNew = NT > 1 || LAYOUT == kPagedPairs;
+  constexpr int kPoolBs = LAYOUT == kPagedPairs ? BS / 2 : BS;  // block size of the pool
+  if constexpr (kStoreNew) store_new_rows_of_empty<D, kPoolBs, kThreads>(a, prefix, batch);
   if (u_begin >= u_end) return;  // uniform: this CTA has no units
 
   [[maybe_unused]] MmaConsumer<D, BS, 1> mc;  // one 8-column tile per warp
@@ -852,6 +859,17 @@ __global__ void __launch_bounds__(kThreads, kStreamCtasPerSm)
       const int nphys = LAYOUT == kPagedPairs
                             ? (effective_len(__ldg(a.seq_lens + b), BS, a, false) + BS / 2 - 1) / (BS / 2)
                             : 0;
+      // fused cache write (kStoreNew): lane p fetches part p of the new row now
+      long long new_slot = -1;
+      uint4 new_part = make_uint4(0u, 0u, 0u, 0u);
+      if constexpr (kStoreNew) {
+        if (a.new_k != nullptr && cnt > 0 && k + cnt == nb) {
+          new_slot = __ldg(a.new_slots + b);
+          if (new_slot >= 0 && lane < 2 * (D / 8))
+            new_part = __ldg((lane < D / 8 ? a.new_k : a.new_v) + (static_cast<size_t>(b) * hkv + h) * (D / 8) +
+                             lane % (D / 8));
+        }
+      }
       for (int base = 0; base < cnt && !stop; base += kPerFetch) {
         int phys = 0;
         if constexpr (LAYOUT == kPaged || LAYOUT == kPagedPairs) {
@@ -873,6 +891,15 @@ __global__ void __launch_bounds__(kThreads, kStreamCtasPerSm)
           const int pb = (LAYOUT == kPaged) ? __shfl_sync(kFull, phys, j)
                                             : (LAYOUT == kPagedPairs ? __shfl_sync(kFull, phys, 2 * j) : 0);
           const int pb1 = (LAYOUT == kPagedPairs) ? __shfl_sync(kFull, phys, 2 * j + 1) : -1;
+          if constexpr (kStoreNew) {
+            if (new_slot >= 0 && base + j == cnt - 1) {  // the (b, h)'s last tile
+              if (lane < 2 * (D / 8)) {
+                store_new_part<D, kPoolBs>(a, new_slot, b, h, lane, new_part);
+                fence_proxy_async_global();  // before lane 0's TMA load of the tile
+              }
+              __syncwarp();
+            }
+          }
           int failed = 0;
           if (lane == 0) {
             const int ii = i + base + j;
@@ -955,8 +982,8 @@ __global__ void __launch_bounds__(kThreads, kStreamCtasPerSm)
       const int last_ii = i + cnt - 1;
       bool patch = false;
       uint4 new_row = make_uint4(0u, 0u, 0u, 0u);
-      // (never with warp pairs: several query tokens, and no cache write)
-      if (grp::kPerGroup == 1 && a.new_k != nullptr && k + cnt == nb && last_ii % kConsumerWarps == warp) {
+      // (warp groups and block pairs: the producer stores the row instead)
+      if (!kStoreNew && a.new_k != nullptr && k + cnt == nb && last_ii % kConsumerWarps == warp) {
         patch = __ldg(a.new_slots + b) >= 0;
         if (patch && lane < 2 * (D / 8)) {
           const uint4* src = (lane < D / 8 ? a.new_k : a.new_v) +
@@ -1385,8 +1412,13 @@ static int launch_stream(const CUtensorMap& map, const DecodeArgs& a, int batch,
   if (rc != PA_OK) return rc;
   PA_CUDA_TRY(launch_pdl(kern, dim3(static_cast<unsigned>(ctas)), dim3(kThreads), smem, st, map, a, batch));
   const int warps = batch * a.qtok * a.num_q_heads;
+  DecodeArgs m = a;
+  if (NT > 1 || LAYOUT == kPagedPairs) {  // the decode kernel stored the new rows already
+    m.new_k = m.new_v = nullptr;
+    m.new_slots = nullptr;
+  }
   PA_CUDA_TRY(launch_pdl(paged_decode_stream_merge_kernel<D, BS>, dim3((warps + 3) / 4), dim3(128), 0, st,
-                         a, batch, ctas));
+                         m, batch, ctas));
   return PA_OK;
 }
 
@@ -1575,11 +1607,11 @@ static int decode_impl(pa_bf16* out, const pa_bf16* q, const pa_bf16* kv_pool,
   a.seg_extra = tc ? tc_decode_segment_extra(bs) : (plan.stream ? kStreamSegExtraTokens / stream_tile(d, bs) : 0);
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   if (fused) {
-    // mma.sync: the decode kernel patches the staged tile, the merge kernel
-    // stores the row; tcgen05: the decode kernel stores the row before the
-    // TMA load of its block; with block pairs or paired warps the cache
-    // write runs first
-    if (plan.stream && !pairs && (tc || a.cols <= kMaxGroup)) {
+    // mma.sync, one warp per block: the decode kernel patches the staged
+    // tile, the merge kernel stores the row; tcgen05, warp groups, block
+    // pairs: the decode kernel's producer stores the row before the TMA
+    // load of its tile; the per-partition grid runs the cache write first
+    if (plan.stream) {
       a.new_k = reinterpret_cast<const uint4*>(new_k);
       a.new_v = reinterpret_cast<const uint4*>(new_v);
       a.new_slots = new_slots;

@@ -152,6 +152,39 @@ __device__ __forceinline__ void block_count_prefix(int* prefix, int* scan, int b
   __syncthreads();
 }
 
+// Fused cache write: part p of request b's newest key / value row of KV
+// head h (p < D/8: 16 bytes of the key, else of the value) into its slot of
+// a pool of PBS-token blocks.  A slot past the pool is flagged and skipped.
+template <int D, int PBS>
+__device__ __forceinline__ void store_new_part(const DecodeArgs& a, long long slot, int b, int h, int p,
+                                               uint4 v) {
+  if (slot >= static_cast<long long>(a.num_blocks) * PBS) {
+    flag_error(a.err, PA_DEVERR_SLOT);
+    return;
+  }
+  const int kv = p / (D / 8), chunk = p % (D / 8);
+  const long long blk = slot / PBS, off = slot - blk * PBS;
+  a.pool_w[(((blk * 2 + kv) * a.num_kv_heads + h) * PBS + off) * (D / 8) + chunk] = v;
+}
+
+// Fused cache write of the requests with no block to attend over (no CTA's
+// range holds them): CTA 0 stores their rows; `prefix` is the balanced
+// schedule's unit prefix table (equal neighbours: no blocks).
+template <int D, int PBS, int NT>
+__device__ __forceinline__ void store_new_rows_of_empty(const DecodeArgs& a, const int* prefix, int batch) {
+  if (a.new_k == nullptr || blockIdx.x != 0) return;
+  const int hkv = a.num_kv_heads;
+  for (int b = threadIdx.x; b < batch; b += NT) {
+    const long long slot = prefix[b + 1] == prefix[b] ? __ldg(a.new_slots + b) : -1;
+    if (slot < 0) continue;
+    for (int h = 0; h < hkv; ++h)
+      for (int p = 0; p < 2 * (D / 8); ++p) {
+        const uint4* src = (p < D / 8 ? a.new_k : a.new_v) + (static_cast<size_t>(b) * hkv + h) * (D / 8) + p % (D / 8);
+        store_new_part<D, PBS>(a, slot, b, h, p, __ldg(src));
+      }
+  }
+}
+
 // Host side of the balanced schedule, shared by the decode translation units.
 // The merge kernel of the balanced schedule for `ctas` persistent CTAs
 // (defined with the mma.sync kernels).

@@ -189,21 +189,6 @@ __device__ __forceinline__ float warp_columns(float (&v)[kTcHalf], int lane) {
   return v[0];
 }
 
-// Fused cache write: part p of request b's newest key / value row of KV
-// head h (p < D/8: 16 bytes of the key, else of the value) into its slot of
-// the pool.  A slot past the pool is flagged and skipped.
-template <int D, int BS>
-__device__ __forceinline__ void store_new_part(const DecodeArgs& a, long long slot, int b, int h, int p,
-                                               uint4 v) {
-  if (slot >= static_cast<long long>(a.num_blocks) * BS) {
-    flag_error(a.err, PA_DEVERR_SLOT);
-    return;
-  }
-  const int kv = p / (D / 8), chunk = p % (D / 8);
-  const long long blk = slot / BS, off = slot - blk * BS;
-  a.pool_w[(((blk * 2 + kv) * a.num_kv_heads + h) * BS + off) * (D / 8) + chunk] = v;
-}
-
 template <int D, int BS, int NH>
 __global__ void __launch_bounds__(tc_threads<NH>(), 1)
     paged_decode_tc_kernel(const __grid_constant__ CUtensorMap kv_map, const __grid_constant__ CUtensorMap q_map,
@@ -307,19 +292,9 @@ __global__ void __launch_bounds__(tc_threads<NH>(), 1)
     }
     v -= kk - nreal + 1;  // the last real block of this (b, h)
   }
-  // fused cache write for requests with no block to attend over: no CTA's
-  // range holds them, so CTA 0 stores their rows (nothing reads them here)
-  if (a.new_k != nullptr && blockIdx.x == 0) {
-    for (int b = threadIdx.x; b < batch; b += kThreads) {
-      const long long slot = prefix[b + 1] == prefix[b] ? __ldg(a.new_slots + b) : -1;
-      if (slot < 0) continue;
-      for (int h = 0; h < hkv; ++h)
-        for (int p = 0; p < 2 * (D / 8); ++p) {
-          const uint4* src = (p < D / 8 ? a.new_k : a.new_v) + (static_cast<size_t>(b) * hkv + h) * (D / 8) + p % (D / 8);
-          store_new_part<D, BS>(a, slot, b, h, p, __ldg(src));
-        }
-    }
-  }
+  // fused cache write for requests with no block to attend over (nothing
+  // reads their rows here)
+  store_new_rows_of_empty<D, BS, kThreads>(a, prefix, batch);
   fence_proxy_async_smem();  // the ring's generic writes above, TMA writes below
   tc::fence_before_sync();
   __syncthreads();

@@ -224,10 +224,8 @@ class PagedDecodeCache:
 
     def launches_per_step(self, npairs):
         """Kernels this library launches for one step."""
-        # the cache write is fused into the balanced decode, except for pools of
-        # 16-token blocks with head dim 64 (two blocks per tile) and groups above
-        # 8 at head dim 64 (paired warps): then it runs first
-        fused = (self.partition_tokens == 0 and self.variant == PA_DECODE_AUTO and self.schedule == "balanced"
-                 and not (self.d == 64 and self.bs == 16) and (self.hq // self.hkv <= 8 or self.d == 128))
+        # the cache write is fused into the balanced decode; on the
+        # per-partition grid (or with explicit choices) it runs first
+        fused = self.partition_tokens == 0 and self.variant == PA_DECODE_AUTO and self.schedule == "balanced"
         cache_write = 0 if fused else 1
         return (1 if npairs else 0) + cache_write + 1 + (1 if self.num_partitions > 1 else 0)

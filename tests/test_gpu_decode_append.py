@@ -26,11 +26,12 @@ def bits(t):
     ([700, 1, 2049, 64, 300, 1500, 17, 1024], 32, 8, 128, 16),   # balanced schedule
     ([900, 33, 5, 2047, 400], 16, 4, 64, 32),                      # balanced, other shape
     ([3, 20, 1], 4, 4, 64, 16),                                    # little work: per-partition grid
-    ([900, 33, 5, 2047, 400, 1600, 2500, 3000], 16, 4, 64, 16),   # balanced on block pairs: write, then decode
+    ([900, 33, 5, 2047, 400, 1600, 2500, 3000], 16, 4, 64, 16),   # balanced on block pairs: stored before the TMA load
     ([700, 1, 2049, 64, 300, 1500, 17, 1024], 32, 2, 128, 16),    # group 16 (tcgen05): stored before the TMA load
     ([700, 1, 2049, 64, 300, 1500, 17, 1024], 48, 2, 128, 32),    # group 24 (tcgen05, two halves), bs32
     ([900, 33, 5, 2047, 400, 128, 127, 129], 64, 4, 128, 16),     # group 16, tile edges
-    ([700, 1, 2049, 64, 300, 1500, 17, 1024], 32, 2, 64, 16),     # group 16 at head dim 64 (paired warps): write, then decode
+    ([700, 1, 2049, 64, 300, 1500, 17, 1024], 32, 2, 64, 16),     # group 16 at head dim 64 (paired warps, pairs)
+    ([700, 1, 2049, 64, 300, 1500, 17, 1024], 64, 2, 64, 32),     # group 32 at head dim 64 (four warps per block)
     ([int(x) for x in np.random.default_rng(67).integers(1, 30, size=4200)], 32, 2, 64, 16),  # 4200 requests: tcgen05
 ])
 def test_append_equals_separate_calls(lens, hq, hkv, d, bs):
@@ -88,13 +89,14 @@ def test_append_equals_separate_calls(lens, hq, hkv, d, bs):
         assert err.mean() <= 1e-3 and (err <= 1e-2 + 2.0 ** -8 * (11.0 + np.abs(want))).all()
 
 
-@pytest.mark.parametrize("hq", [8, 32])
-def test_append_with_empty_requests(hq):
+@pytest.mark.parametrize("hq,d", [(8, 128), (32, 128), (32, 64)])
+def test_append_with_empty_requests(hq, d):
     """Empty requests with and without a slot (one writes into a block no
     request holds: only the cache write touches it); group 4 on mma.sync,
-    group 16 on the tcgen05 consumer."""
+    group 16 on the tcgen05 consumer, group 16 at head dim 64 on paired
+    warps over block pairs."""
     dev = torch.device("cuda", torch.cuda.current_device())
-    hkv, d, bs = 2, 128, 16
+    hkv, bs = 2, 16
     lens = [0, 1500, 0, 2000] * 8  # 32 requests, enough work for the balanced schedule
     nb = sum(-(-n // bs) for n in lens) + 4
     a = pk.PaAlloc(nb, bs)
