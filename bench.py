@@ -542,6 +542,18 @@ def run_gpu(args):
     del arm, cache
     torch.cuda.empty_cache()
 
+    # ---- wide GQA groups (the tcgen05 consumer) against mma.sync on the same
+    # lengths: decode + merge back to back (one GPU, default workload only)
+    wide = []
+    if world == 1 and args.workload == "llama8b" and not args.no_workloads:
+        peaks = load_peaks()
+        for row in variant_times(iters=20, hkvs=[(8, 128)], groups=[16, 32]):
+            row.pop("cuda_core_us", None)
+            row.pop("cuda_core_gbs", None)
+            row["tcgen05_frac_of_hbm_peak"] = round(row["tcgen05_gbs"] / peaks["hbm_gbs"], 4)
+            row["default_variant"] = "tcgen05"
+            wide.append(row)
+
     # ---- the other workloads, device-timed (one GPU, default workload only)
     others = {}
     if world == 1 and args.workload == "llama8b" and not args.no_workloads:
@@ -621,6 +633,8 @@ def run_gpu(args):
         }
         if others:
             line["workloads"] = others
+        if wide:
+            line["wide_columns"] = wide
         if world == 1 and not args.no_cpu_baseline:
             line["cpu_baseline"] = cpu_baseline(args.workload, args.cpu_seconds)
         print(json.dumps(line), flush=True)
@@ -955,11 +969,12 @@ def study_multi_token(iters=30):
     assert pk.pa_device_error() == 0
 
 
-def study_variants(iters=20, hkvs=None, groups=None, only=None):
+def variant_times(iters=20, hkvs=None, groups=None, only=None):
     """The three consumers across GQA group sizes: pa_decode on the llama8b
     lengths and shuffled pool, Hkv in {8, 32}, head dim 128 and (Hkv 8) 64,
     groups 1, 2, 4, 8, 16, 32 -- mma.sync and tcgen05 for every group, CUDA
-    cores for 1, 2, 4; CUDA events over back-to-back launches."""
+    cores for 1, 2, 4; CUDA events over back-to-back launches.  Yields one
+    dict per (Hkv, head dim, group)."""
     import torch
 
     import paged_kv_cache_354_b200 as pk
@@ -1004,13 +1019,17 @@ def study_variants(iters=20, hkvs=None, groups=None, only=None):
                 e1.record()
                 torch.cuda.synchronize()
                 res[name] = e0.elapsed_time(e1) / iters * 1e3
-            print(json.dumps({"study": "variants", "workload": "llama8b lengths", "num_kv_heads": hkv,
-                              "head_dim": d, "group": g, **{f"{k}_us": round(v, 1) for k, v in res.items()},
-                              **{f"{k}_gbs": round(nbytes / v / 1e3, 1) for k, v in res.items()},
-                              "iters": iters}), flush=True)
+            yield {"workload": "llama8b lengths", "num_kv_heads": hkv, "head_dim": d, "group": g,
+                   **{f"{k}_us": round(v, 1) for k, v in res.items()},
+                   **{f"{k}_gbs": round(nbytes / v / 1e3, 1) for k, v in res.items()}, "iters": iters}
         del pool
         torch.cuda.empty_cache()
     assert pk.pa_device_error() == 0
+
+
+def study_variants(iters=20, hkvs=None, groups=None, only=None):
+    for row in variant_times(iters, hkvs, groups, only):
+        print(json.dumps({"study": "variants", **row}), flush=True)
 
 
 def study_read_bandwidth(iters=20):
