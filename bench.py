@@ -543,8 +543,9 @@ def run_gpu(args):
     torch.cuda.empty_cache()
 
     # ---- wide GQA groups (the tcgen05 consumer) against mma.sync on the same
-    # lengths: decode + merge back to back (one GPU, default workload only)
-    wide = []
+    # lengths, and multi-token decode with T = 1, 2, 4 query tokens: decode +
+    # merge back to back (one GPU, default workload only)
+    wide, multi = [], []
     if world == 1 and args.workload == "llama8b" and not args.no_workloads:
         peaks = load_peaks()
         for row in variant_times(iters=20, hkvs=[(8, 128)], groups=[16, 32]):
@@ -553,6 +554,7 @@ def run_gpu(args):
             row["tcgen05_frac_of_hbm_peak"] = round(row["tcgen05_gbs"] / peaks["hbm_gbs"], 4)
             row["default_variant"] = "tcgen05"
             wide.append(row)
+        multi = list(multi_token_times())
 
     # ---- the other workloads, device-timed (one GPU, default workload only)
     others = {}
@@ -635,6 +637,8 @@ def run_gpu(args):
             line["workloads"] = others
         if wide:
             line["wide_columns"] = wide
+        if multi:
+            line["multi_token"] = multi
         if world == 1 and not args.no_cpu_baseline:
             line["cpu_baseline"] = cpu_baseline(args.workload, args.cpu_seconds)
         print(json.dumps(line), flush=True)
@@ -927,10 +931,11 @@ def study_page_table(iters=30, names=("llama8b", "mixed", "long")):
     assert pk.pa_device_error() == 0
 
 
-def study_multi_token(iters=30):
+def multi_token_times(iters=30):
     """pa_decode_multi at the llama8b shape for T = 1, 2, 4 causal query
     tokens per request (speculative verification): KV bytes stay the same,
-    the tensor-core tile widens from 4 to 16 (token, head) columns."""
+    the tensor-core tile widens from 4 to 16 (token, head) columns.  Yields
+    one dict per T."""
     import torch
 
     import paged_kv_cache_354_b200 as pk
@@ -961,12 +966,18 @@ def study_multi_token(iters=30):
         torch.cuda.synchronize()
         us = e0.elapsed_time(e1) / iters * 1e3
         extra_qo = 2 * len(ids) * (T - 1) * cache.hq * cache.d * 2
-        print(json.dumps({"study": "multi_token", "workload": "llama8b", "query_tokens": T,
-                          "columns_per_kv_head": T * cache.hq // cache.hkv, "us": round(us, 2),
-                          "gbs": round((nbytes + extra_qo) / us / 1e3, 1),
-                          "frac_of_hbm_peak": round((nbytes + extra_qo) / us / 1e3 / load_peaks()["hbm_gbs"], 4),
-                          "tokens_per_s": round(len(ids) * T / us * 1e6, 1)}), flush=True)
+        yield {"workload": "llama8b", "query_tokens": T, "columns_per_kv_head": T * cache.hq // cache.hkv,
+               "us": round(us, 2), "gbs": round((nbytes + extra_qo) / us / 1e3, 1),
+               "frac_of_hbm_peak": round((nbytes + extra_qo) / us / 1e3 / load_peaks()["hbm_gbs"], 4),
+               "tokens_per_s": round(len(ids) * T / us * 1e6, 1)}
+    del cache
+    torch.cuda.empty_cache()
     assert pk.pa_device_error() == 0
+
+
+def study_multi_token(iters=30):
+    for row in multi_token_times(iters):
+        print(json.dumps({"study": "multi_token", **row}), flush=True)
 
 
 def variant_times(iters=20, hkvs=None, groups=None, only=None):
