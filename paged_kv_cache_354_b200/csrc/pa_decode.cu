@@ -1604,7 +1604,7 @@ static int decode_impl(pa_bf16* out, const pa_bf16* q, const pa_bf16* kv_pool,
   a.pool_w = reinterpret_cast<uint4*>(const_cast<pa_bf16*>(kv_pool));
   // overhead-weighted split of the balanced schedule (virtual units per
   // (request, KV head), in the kernel's tiles)
-  a.seg_extra = tc ? tc_decode_segment_extra(bs) : (plan.stream ? kStreamSegExtraTokens / stream_tile(d, bs) : 0);
+  a.seg_extra = tc ? tc_decode_segment_extra(bs, a.cols) : (plan.stream ? kStreamSegExtraTokens / stream_tile(d, bs) : 0);
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   if (fused) {
     // mma.sync, one warp per block: the decode kernel patches the staged

@@ -193,7 +193,7 @@ int launch_stream_merge(int d, int bs, const DecodeArgs& a, int batch, int ctas,
 // block_size 16/32; launches the decode kernel and the merge.
 int tc_decode_supported(int d, int bs, int cols);
 // Virtual units per (request, KV head) the tcgen05 consumer's split adds.
-int tc_decode_segment_extra(int bs);
+int tc_decode_segment_extra(int bs, int cols);
 int launch_tc_decode(const DecodeArgs& a, const void* kv_pool, int batch, int d, int bs, int num_blocks,
                      int ctas, cudaStream_t st);
 

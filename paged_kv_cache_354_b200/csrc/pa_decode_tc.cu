@@ -773,8 +773,16 @@ int launch_tc_cols(const CUtensorMap& kv_map, const CUtensorMap& q_map, const De
 #ifndef PA_TC_SEG_EXTRA_TOKENS
 #define PA_TC_SEG_EXTRA_TOKENS 192
 #endif
+// ... and with two 16-column halves (an epilogue per half, twice the MMA
+// columns): group 32 at the llama8b lengths, 192 / 256 / 320 / 384 tokens:
+// 122.4 / 120.5 / 120.6 / 121.2 us (decode + merge)
+#ifndef PA_TC_SEG_EXTRA_TOKENS_TWO_HALVES
+#define PA_TC_SEG_EXTRA_TOKENS_TWO_HALVES 256
+#endif
 
-int tc_decode_segment_extra(int bs) { return PA_TC_SEG_EXTRA_TOKENS / bs; }
+int tc_decode_segment_extra(int bs, int cols) {
+  return (cols > kTcHalf ? PA_TC_SEG_EXTRA_TOKENS_TWO_HALVES : PA_TC_SEG_EXTRA_TOKENS) / bs;
+}
 
 int tc_decode_supported(int d, int bs, int cols) {
   return (d == 64 || d == 128) && (bs == 16 || bs == 32) && cols >= 1 && cols <= kTcMaxCols;
