@@ -819,8 +819,8 @@ __global__ void __launch_bounds__(kThreads, kStreamCtasPerSm)
     *abort_flag = 0;
     fence_barrier_init();
   }
-  pdl_trigger();
   pdl_wait();  // every global access below comes after the previous grid
+  pdl_trigger();  // after the wait: the merge reads inputs before its own
   block_count_prefix<BS, kThreads>(prefix, reinterpret_cast<int*>(smem + sm::kScan), batch, a,
                          blockIdx.x == 0);
   if (blockIdx.x == 0)
@@ -1092,44 +1092,68 @@ __global__ void __launch_bounds__(kThreads, kStreamCtasPerSm)
 // CTAs c_first..c_last is merged from their partial slots (slot 0 when the
 // (b, h) is the CTA's first segment, else slot 1).  CTAs with an empty range
 // (more CTAs than units) wrote nothing and are skipped.  Requests of length
-// 0 get zeros here.  Two dependent memory rounds per warp: the prefix sums,
-// then (m, l) and the O row slice of up to 8 covering CTAs at once.
+// 0 get zeros here.
+//
+// What does not depend on the decode kernel's output is done before the
+// grid dependency wait, while the decode still streams: up to
+// kMergeLocalPrefix requests, the block-count prefix sums (from the lengths,
+// with the decode kernel's own arithmetic), and the loads of the new
+// tokens' K/V rows of the fused cache write.  Those are inputs no kernel of
+// the call writes, and the decode kernel lets this grid launch only after
+// its own wait, so whatever wrote them has finished.  After the wait one
+// dependent memory round per warp is left: (m, l) and the O row slice of up
+// to 8 covering CTAs at once (larger batches first read the decode kernel's
+// copy of the prefix sums).
+constexpr int kMergeLocalPrefix = 512;
+
 template <int D, int BS>
 __global__ void __launch_bounds__(128) paged_decode_stream_merge_kernel(const DecodeArgs a,
                                                                         int batch, int ctas) {
   constexpr int kPer = D / 32;
   constexpr int kUnroll = 8;
+  __shared__ int s_prefix[kMergeLocalPrefix + 1];
+  __shared__ int s_scan[128 + 1];
   pdl_trigger();
-  pdl_wait();
+  const bool local = batch <= kMergeLocalPrefix;  // uniform
+  if (local) block_count_prefix<BS, 128>(s_prefix, s_scan, batch, a, false);
   const int gw = blockIdx.x * 4 + (threadIdx.x >> 5);  // (request, token, query head)
   const int lane = threadIdx.x & 31;
   const int hkv = a.num_kv_heads;
   const int g = a.group;
   const int per_req = a.qtok * a.num_q_heads;
-  if (gw >= batch * per_req) return;
-  const int b = gw / per_req;
+  const bool live = gw < batch * per_req;
+  const int b = live ? gw / per_req : 0;
   const int t = (gw - b * per_req) / a.num_q_heads;
   const int qh = gw - b * per_req - t * a.num_q_heads;  // query head
   const int h = qh / g;                                 // its KV head
   const int j = t * g + (qh - h * g);                   // its column in the (token, head) tile
   const int cols = a.cols;
-  if (a.new_k != nullptr && t == 0 && qh == h * g && lane < 2 * (D / 8)) {
-    // fused cache write: the decode kernel has finished reading the pool,
-    // so request b's new K/V row for KV head h lands in its slot now
-    const long long slot = __ldg(a.new_slots + b);
+  // fused cache write: lane p of the KV head's first warp fetches part p of
+  // request b's new K/V row now and stores it once the decode kernel has
+  // finished reading the pool
+  const bool writer = live && a.new_k != nullptr && t == 0 && qh == h * g && lane < 2 * (D / 8);
+  long long new_slot = -1;
+  uint4 new_part = make_uint4(0u, 0u, 0u, 0u);
+  if (writer) {
+    new_slot = __ldg(a.new_slots + b);
+    new_part = __ldg((lane < D / 8 ? a.new_k : a.new_v) + (static_cast<size_t>(b) * hkv + h) * (D / 8) +
+                     lane % (D / 8));
+  }
+  pdl_wait();
+  if (!live) return;
+  if (writer) {
     const long long nslots = static_cast<long long>(a.num_blocks) * BS;
-    if (slot >= nslots) {
+    if (new_slot >= nslots) {
       if (lane == 0) flag_error(a.err, PA_DEVERR_SLOT);
-    } else if (slot >= 0) {
+    } else if (new_slot >= 0) {
       const int kv = lane / (D / 8);
       const int chunk = lane % (D / 8);
-      const long long blk = slot / BS;
-      const long long off = slot - blk * BS;
-      const uint4* src = (kv ? a.new_v : a.new_k) + (static_cast<size_t>(b) * hkv + h) * (D / 8) + chunk;
-      a.pool_w[(((blk * 2 + kv) * hkv + h) * BS + off) * (D / 8) + chunk] = __ldg(src);
+      const long long blk = new_slot / BS;
+      const long long off = new_slot - blk * BS;
+      a.pool_w[(((blk * 2 + kv) * hkv + h) * BS + off) * (D / 8) + chunk] = new_part;
     }
   }
-  const int* prefix = a.stream_prefix;
+  const int* prefix = local ? s_prefix : a.stream_prefix;
   const int pb0 = prefix[b], pb1 = prefix[b + 1], pall = prefix[batch];
   const int nbu = pb1 - pb0;                          // work units of each (b, h)
   const int nb = nbu > 0 ? nbu - a.seg_extra : 0;     // of which real blocks

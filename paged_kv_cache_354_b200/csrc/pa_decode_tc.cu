@@ -265,8 +265,8 @@ __global__ void __launch_bounds__(tc_threads<NH>(), 1)
     tc::tmem_alloc(smem_u32(tmem_slot), G::kTmemCols);
     tc::tmem_relinquish();
   }
-  pdl_trigger();
   pdl_wait();  // every global access below comes after the previous grid
+  pdl_trigger();  // after the wait: the merge reads inputs before its own
 
   // per-request block-count prefix sums, in the still idle K ring
   int* prefix = reinterpret_cast<int*>(smem + G::kK);

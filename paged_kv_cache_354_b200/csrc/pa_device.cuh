@@ -37,7 +37,12 @@ __device__ __forceinline__ uint64_t globaltimer_ns() {
 // the kernel before it.  The rule that keeps this safe: a kernel calls
 // pdl_wait() before its first global-memory access (read or write); that
 // wait returns once the preceding grid has completed and its writes are
-// visible.  pdl_trigger() lets the next kernel launch early.
+// visible.  pdl_trigger() lets the next kernel launch early.  One exception:
+// the balanced schedule's merge kernel reads inputs of the call (lengths,
+// the new tokens' rows) before its wait; the decode kernels that precede it
+// trigger only after their own wait, so every earlier writer has finished
+// by the time the merge grid launches, and the decode kernels write none of
+// those inputs.
 __device__ __forceinline__ void pdl_wait() { cudaGridDependencySynchronize(); }
 __device__ __forceinline__ void pdl_trigger() { cudaTriggerProgrammaticLaunchCompletion(); }
 
