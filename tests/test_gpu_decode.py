@@ -176,6 +176,17 @@ def test_balanced_schedule_at_its_batch_limit(hq, variant):
     check_short(lens, hq, 2, 128, 16, seed=63, variant=variant)
 
 
+@pytest.mark.parametrize("batch", [512, 513])
+@pytest.mark.parametrize("hq,variant", [(8, "mma"), (32, "tcgen05"), (64, "tcgen05")])
+def test_merge_prefix_sums_either_side_of_its_local_limit(batch, hq, variant):
+    """The merge kernel of the balanced schedule computes the block-count
+    prefix sums itself for up to 512 requests and reads the decode kernel's
+    copy above that: both sides of the limit, with many (request, head) pairs
+    cut between CTAs and some empty requests."""
+    lens = list(np.random.default_rng(66 + batch).integers(0, 200, size=batch))
+    check_short(lens, hq, 2, 128, 16, seed=66 + batch, variant=variant)
+
+
 @pytest.mark.parametrize("hq,d,bs", [(32, 128, 16), (32, 64, 16), (48, 128, 32)])
 def test_wide_groups_above_the_batch_limit(hq, d, bs):
     """More than 8 columns with more than 4096 requests: the default variant

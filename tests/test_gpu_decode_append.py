@@ -33,6 +33,10 @@ def bits(t):
     ([700, 1, 2049, 64, 300, 1500, 17, 1024], 32, 2, 64, 16),     # group 16 at head dim 64 (paired warps, pairs)
     ([700, 1, 2049, 64, 300, 1500, 17, 1024], 64, 2, 64, 32),     # group 32 at head dim 64 (four warps per block)
     ([int(x) for x in np.random.default_rng(67).integers(1, 30, size=4200)], 32, 2, 64, 16),  # 4200 requests: tcgen05
+    # 512 / 513 requests: the merge kernel (which stores the new rows on this
+    # path) computes the prefix sums itself, or reads the decode kernel's copy
+    ([int(x) for x in np.random.default_rng(68).integers(1, 200, size=512)], 8, 2, 128, 16),
+    ([int(x) for x in np.random.default_rng(69).integers(1, 200, size=513)], 8, 2, 128, 16),
 ])
 def test_append_equals_separate_calls(lens, hq, hkv, d, bs):
     dev = torch.device("cuda", torch.cuda.current_device())
@@ -79,12 +83,12 @@ def test_append_equals_separate_calls(lens, hq, hkv, d, bs):
     assert np.array_equal(bits(pool_b), want_pool)
     t_ref, l_ref = workloads.block_tables(ref, ids, mb)
     want = opa.decode(q.double().cpu().numpy(), u16_to_f64(want_pool), t_ref, l_ref, scale)
-    if len(lens) <= 4096:
+    if len(lens) <= 64:
         compare(out_b.double().cpu().numpy(), want)
     else:
-        # thousands of requests of a few positions: the bf16 probabilities and
-        # output can move an element by 2^-8 (|v - out| spread + |out|) beyond
-        # 1e-2 (tests/test_gpu_decode.py, check_short); |v| < ~5.5 here
+        # hundreds of requests, some of a few positions: the bf16 probabilities
+        # and output can move an element by 2^-8 (|v - out| spread + |out|)
+        # beyond 1e-2 (tests/test_gpu_decode.py, check_short); |v| < ~5.5 here
         err = np.abs(out_b.double().cpu().numpy() - want)
         assert err.mean() <= 1e-3 and (err <= 1e-2 + 2.0 ** -8 * (11.0 + np.abs(want))).all()
 
