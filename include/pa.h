@@ -23,6 +23,10 @@
  *  - Kernel calls are asynchronous on `stream` (a cudaStream_t / CUstream
  *    handle, NULL = legacy default stream).  Argument errors are reported
  *    before anything is launched.  A launch failure returns PA_ERR_CUDA.
+ *    The kernels are launched with programmatic stream serialisation: a
+ *    kernel may start while the one before it on the stream finishes, and
+ *    waits for that kernel's completion before it touches any memory the
+ *    call's arguments name, so stream order holds as usual.
  *  - Device-side checks (block ids outside the pool, a slot outside the
  *    pool, a length beyond the block table, a pipeline wait that timed out)
  *    never trap: the kernel skips the offending access and records a code
