@@ -46,3 +46,30 @@ def test_memory_waste_study_lines():
     assert by_name["mixed"]["contiguous_waste_frac"] > 0.6 > 0.05 > by_name["mixed"]["paged_internal_waste_frac"]
     # beams sharing their prefix hold far fewer physical slots than tokens
     assert by_name["beam"]["paged_physical_over_tokens"] < 0.5
+
+
+def test_committed_profiles_cite_one_capture():
+    """The DRAM traffic that bench.py reports as roofline.traffic comes from
+    profiles/paged_decode_traffic.json, and only while the decode sources hash
+    to the digest stored there; every ncu summary under profiles/ names the
+    sources it was captured on by that same digest, so the committed
+    evidence is one capture of one set of sources."""
+    import re
+
+    with open(os.path.join(ROOT, "profiles", "paged_decode_traffic.json")) as f:
+        rec = json.load(f)
+    digests = {e["source_sha256"] for e in rec.values()}
+    assert len(digests) == 1
+    (digest,) = digests
+    for e in rec.values():
+        assert e["dram_read_bytes"] + e["dram_write_bytes"] == e["dram_bytes_per_launch"] > 0
+    cited = {}
+    for name in sorted(os.listdir(os.path.join(ROOT, "profiles"))):
+        if name.endswith(".md"):
+            with open(os.path.join(ROOT, "profiles", name)) as f:
+                found = set(re.findall(r"`([0-9a-f]{64})`", f.read()))
+            if found:
+                cited[name] = found
+    assert cited, "no summary names its sources"
+    for name, found in cited.items():
+        assert found == {digest}, name
